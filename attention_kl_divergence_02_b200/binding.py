@@ -1,0 +1,177 @@
+"""ctypes binding of libstreamkl (include/streamkl.h).
+
+Argument marshalling only: torch tensors are turned into device pointers and the CUDA
+stream handle, and every step of the computation runs in the library's kernels.  The
+library is loaded on first use; if it is missing or fails to load this raises, there is
+no other implementation to fall back to.
+
+Low-level functions carry the C names and arguments (pointers may be ints or tensors).
+``fwd``/``bwd`` are conveniences that allocate outputs with torch (device memory is
+torch's job; the library allocates nothing).
+"""
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libstreamkl.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_CUDA = 3
+ERR_TIMEOUT = 4
+
+EXPORTS = (
+    "streamkl_fwd",
+    "streamkl_bwd",
+    "streamkl_bwd_workspace_bytes",
+    "streamkl_status_string",
+    "streamkl_device_status",
+    "streamkl_last_cuda_error",
+    "streamkl_version",
+)
+
+_lib = None
+
+
+class StreamKLError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = "%s: %s" % (where, status_string(status))
+        if status == ERR_CUDA:
+            msg += " (%s)" % last_cuda_error()
+        super().__init__(msg)
+
+
+def load(path=None):
+    """Load the shared library (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError("libstreamkl.so not built at %s (run python -m "
+                          "attention_kl_divergence_02_b200.build)" % p)
+    lib = ctypes.CDLL(p)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.streamkl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+    lib.streamkl_fwd.restype = i
+    lib.streamkl_bwd.argtypes = ([i, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                  vp, vp, vp, sz, vp])
+    lib.streamkl_bwd.restype = i
+    lib.streamkl_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.streamkl_bwd_workspace_bytes.restype = sz
+    lib.streamkl_status_string.argtypes = [i]
+    lib.streamkl_status_string.restype = ctypes.c_char_p
+    lib.streamkl_device_status.argtypes = [vp]
+    lib.streamkl_device_status.restype = i
+    lib.streamkl_last_cuda_error.argtypes = []
+    lib.streamkl_last_cuda_error.restype = ctypes.c_char_p
+    lib.streamkl_version.argtypes = []
+    lib.streamkl_version.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ C-named calls
+def streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, kl, lse1, lse2, stream=None):
+    return load().streamkl_fwd(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), B, Hq, Hkv, NQ, NK, d,
+                               float(scale), int(bool(causal)), _ptr(kl), _ptr(lse1), _ptr(lse2),
+                               _stream(stream))
+
+
+def streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale, causal,
+                 dq, dk, workspace, workspace_bytes, stream=None):
+    return load().streamkl_bwd(int(mode), _ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(kl),
+                               _ptr(lse1), _ptr(lse2), _ptr(dkl), B, Hq, Hkv, NQ, NK, d,
+                               float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
+                               _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def streamkl_bwd_workspace_bytes(B, Hq, NQ, d):
+    return load().streamkl_bwd_workspace_bytes(B, Hq, NQ, d)
+
+
+def streamkl_device_status(stream=None):
+    return load().streamkl_device_status(_stream(stream))
+
+
+def status_string(status):
+    return load().streamkl_status_string(int(status)).decode()
+
+
+def last_cuda_error():
+    return load().streamkl_last_cuda_error().decode()
+
+
+def version():
+    return load().streamkl_version()
+
+
+# ------------------------------------------------------------------ conveniences
+def _dims(q1, k1):
+    B, Hq, NQ, d = q1.shape
+    _, Hkv, NK, _ = k1.shape
+    return B, Hq, Hkv, NQ, NK, d
+
+
+def _check_inputs(q1, k1, q2, k2):
+    import torch
+    for t in (q1, k1, q2, k2):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous bf16 CUDA tensors")
+    if q1.shape != q2.shape or k1.shape != k2.shape or q1.dim() != 4 or k1.dim() != 4:
+        raise ValueError("q1/q2 must be [B,Hq,NQ,d], k1/k2 [B,Hkv,NK,d]")
+
+
+def fwd(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
+    """Returns (kl, lse1, lse2), fp32 [B,Hq,NQ].  Pass k2 = k1 (same tensor) for shared keys."""
+    import torch
+    _check_inputs(q1, k1, q2, k2)
+    B, Hq, Hkv, NQ, NK, d = _dims(q1, k1)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = tuple(torch.empty((B, Hq, NQ), dtype=torch.float32, device=q1.device) for _ in range(3))
+    rc = streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, *out, stream=stream)
+    if rc != OK:
+        raise StreamKLError(rc, "streamkl_fwd")
+    return out
+
+
+def bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, scale=None, causal=False, out=None,
+        workspace=None, stream=None):
+    """Returns (dq, dk) of the free distribution: mode 1 -> (dQ2, dK2), mode 2 -> (dQ1, dK1)."""
+    import torch
+    _check_inputs(q1, k1, q2, k2)
+    B, Hq, Hkv, NQ, NK, d = _dims(q1, k1)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = (torch.empty_like(q1), torch.empty_like(k1))
+    nbytes = streamkl_bwd_workspace_bytes(B, Hq, NQ, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16) // 4, dtype=torch.float32, device=q1.device)
+    rc = streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
+                      causal, out[0], out[1], workspace, workspace.numel() * workspace.element_size(),
+                      stream=stream)
+    if rc != OK:
+        raise StreamKLError(rc, "streamkl_bwd")
+    return out

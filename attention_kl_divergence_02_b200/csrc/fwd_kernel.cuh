@@ -1,0 +1,335 @@
+// fwd_kernel.cuh -- StreamKL forward on sm_100a.
+//
+// One CTA owns 256 query rows of one (batch, query head): two 128-row tiles t = 0, 1.
+// Key tiles of 128 keys stream through a ring of shared-memory slots filled by TMA.  For
+// every key tile the tensor core computes S1 = Q1 K1^T and S2 = Q2 K2^T for both query
+// tiles into TMEM (fp32, lane = query row, column = key), and one 128-thread warpgroup per
+// query tile (one thread per row) folds the tile into the row's five running scalars
+//   m1, l1, m2, l2, acc
+// (StreamKL technical summary, gist.science, Portuguese, "1. Formulação Online (Passagem
+// Forward)"), rescaling l1, acc and l2 by 2^(m_old - m_new) whenever a maximum grows (the
+// online correction of the FlashAttention lecture notes, hackmd, "4. Flash Attention 的核心
+// 數學重構").  At the end it writes KL = acc/l1 + LSE2 - LSE1 and both LSEs.  Causal key
+// tiles past the diagonal are never loaded or multiplied.
+//
+// Roles (384 threads):  warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
+// warps 2-3 idle, warps 4-7 = statistics warpgroup of tile 0, warps 8-11 = tile 1.
+// Warp w may touch TMEM lanes 32*(w%4) .. 32*(w%4)+31, so each statistics warp owns the
+// 32 rows that live in its lane quarter.
+//
+// Scores are kept in base-2 units: u = s_raw * scale * log2(e), where s_raw = <q, k>.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace skl {
+
+struct FwdParams {
+    int B, Hq, Hkv, NQ, NK;
+    int causal;
+    int n_qblk;    // ceil(NQ / 256)
+    float sl2;     // scale * log2(e)
+    float scale;
+    float* kl;
+    float* lse1;
+    float* lse2;
+};
+
+constexpr int kFwdThreads = 384;
+
+template <int D>
+struct FwdCfg {
+    static constexpr int kTile = 128 * D * 2;       // bytes of one 128-row bf16 tile
+    static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
+    static constexpr int kBox = 128 * 128;          // bytes of one box: 128 rows x 128 bytes
+    static constexpr int kSlots = (D == 128) ? 3 : 6;
+    static constexpr int kQ1 = 0;                   // Q1 tile t at kQ1 + t*kTile
+    static constexpr int kQ2 = 2 * kTile;           // Q2 tile t at kQ2 + t*kTile
+    static constexpr int kK = 4 * kTile;            // key slot s at kK + s*kTile
+    static constexpr int kBar = kK + kSlots * kTile;
+    // barrier indices
+    static constexpr int Q_FULL = 0;                // + t
+    static constexpr int K_FULL = 2;                // + s
+    static constexpr int K_EMPTY = 2 + kSlots;      // + s
+    static constexpr int S_FULL = 2 + 2 * kSlots;   // + t
+    static constexpr int S_FREE = S_FULL + 2;       // + t
+    static constexpr int DONE = S_FREE + 2;
+    static constexpr int kNumBars = DONE + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem address, abort flag
+    static constexpr int kSmem = kMisc + 16 + 1024;     // + slack for 1024-byte alignment
+};
+
+
+// Fold 32 columns of one row into the running scalars.  x = S1 raw scores, y = S2 raw.
+// `valid` has bit k set when column k is a valid key for this row.
+template <bool MASKED>
+__device__ __forceinline__ void fold_chunk(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
+                                           uint32_t valid, float sl2, float& m1, float& l1,
+                                           float& m2, float& l2, float& acc) {
+    float x[32], y[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        x[k] = __uint_as_float(xa[k]);
+        y[k] = __uint_as_float(ya[k]);
+        if (MASKED && !((valid >> k) & 1u)) {
+            x[k] = -INFINITY;
+            y[k] = -INFINITY;
+        }
+    }
+    float mx1 = x[0], mx2 = y[0];
+#pragma unroll
+    for (int k = 1; k < 32; ++k) {
+        mx1 = fmaxf(mx1, x[k]);
+        mx2 = fmaxf(mx2, y[k]);
+    }
+    const float m1n = fmaxf(m1, mx1 * sl2);
+    const float m2n = fmaxf(m2, mx2 * sl2);
+    const float a1 = ex2(m1 - m1n);
+    const float a2 = ex2(m2 - m2n);
+    m1 = m1n;
+    m2 = m2n;
+    float sl1[2] = {0.f, 0.f}, sl2v[2] = {0.f, 0.f}, sac[2] = {0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float e1 = ex2(fmaf(x[k], sl2, -m1n));
+        const float e2 = ex2(fmaf(y[k], sl2, -m2n));
+        float diff = x[k] - y[k];
+        if (MASKED && !((valid >> k) & 1u)) diff = 0.f;
+        sl1[k & 1] += e1;
+        sl2v[k & 1] += e2;
+        sac[k & 1] = fmaf(e1, diff, sac[k & 1]);
+    }
+    l1 = fmaf(l1, a1, sl1[0] + sl1[1]);
+    acc = fmaf(acc, a1, sac[0] + sac[1]);
+    l2 = fmaf(l2, a2, sl2v[0] + sl2v[1]);
+}
+
+template <int D, bool SHARED_K>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
+                    const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
+                    const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(smem);
+    const uint32_t bar0 = sb + C::kBar;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+#define BAR(i) (bar0 + 8u * (uint32_t)(i))
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: heaviest causal query blocks are handed out first
+    const int BH = p.B * p.Hq;
+    const int unit = blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
+    const int qb = p.causal ? (p.n_qblk - 1 - unit) : unit;
+    const int b = bh / p.Hq;
+    const int h = bh % p.Hq;
+    const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
+    const int nkt_all = (p.NK + 127) >> 7;
+    int q0[2], nkt[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        q0[t] = qb * 256 + t * 128;
+        if (q0[t] >= p.NQ) {
+            nkt[t] = 0;
+        } else if (p.causal) {
+            const int last_row = min(q0[t] + 127, p.NQ - 1);
+            nkt[t] = min(nkt_all, (last_row >> 7) + 1);
+        } else {
+            nkt[t] = nkt_all;
+        }
+    }
+    const int ntiles = nkt[1] > 0 ? 2 : 1;
+    const int nj = max(nkt[0], nkt[1]);
+
+    // ---- setup
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(BAR(C::Q_FULL + t), 1);
+            mbar_init(BAR(C::S_FULL + t), 1);
+            mbar_init(BAR(C::S_FREE + t), 128);
+        }
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(BAR(C::K_FULL + s), 1);
+            mbar_init(BAR(C::K_EMPTY + s), 1);
+        }
+        mbar_init(BAR(C::DONE), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ1);
+            tma_prefetch_desc(&tmQ2);
+            tma_prefetch_desc(&tmK1);
+            if (!SHARED_K) tma_prefetch_desc(&tmK2);
+            for (int t = 0; t < ntiles; ++t) {
+                mbar_arrive_expect_tx(BAR(C::Q_FULL + t), 2 * C::kTile);
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_3d(sb + C::kQ1 + t * C::kTile + bx * C::kBox, &tmQ1, BAR(C::Q_FULL + t),
+                                bx * 64, q0[t], bh);
+                    tma_load_3d(sb + C::kQ2 + t * C::kTile + bx * C::kBox, &tmQ2, BAR(C::Q_FULL + t),
+                                bx * 64, q0[t], bh);
+                }
+            }
+            uint32_t it = 0;
+            bool ok = true;
+            for (int j = 0; j < nj && ok; ++j) {
+#pragma unroll
+                for (int w = 0; w < (SHARED_K ? 1 : 2); ++w) {
+                    const uint32_t s = it % C::kSlots;
+                    const uint32_t n = it / C::kSlots;
+                    if (n > 0 && !mbar_wait(BAR(C::K_EMPTY + s), (n - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(BAR(C::K_FULL + s), C::kTile);
+                    const CUtensorMap* map = (w == 0) ? &tmK1 : &tmK2;
+                    for (int bx = 0; bx < C::kBoxes; ++bx)
+                        tma_load_3d(sb + C::kK + s * C::kTile + bx * C::kBox, map, BAR(C::K_FULL + s),
+                                    bx * 64, j * 128, bhk);
+                    ++it;
+                }
+            }
+            // drain: every copy this thread started must land before the CTA exits
+            for (int t = 0; t < ntiles; ++t) drain_wait(BAR(C::Q_FULL + t), 0);
+            for (uint32_t s = 0; s < (uint32_t)C::kSlots; ++s) {
+                if (it > s) {
+                    const uint32_t fills = (it - s - 1) / C::kSlots + 1;
+                    drain_wait(BAR(C::K_FULL + s), (fills - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 0);
+            bool ok = true;
+            for (int t = 0; t < ntiles && ok; ++t) ok = mbar_wait(BAR(C::Q_FULL + t), 0, abort_flag);
+            tc_fence_after();
+            uint32_t it = 0;
+            for (int j = 0; j < nj && ok; ++j) {
+                const uint32_t s1 = it % C::kSlots;
+                if (!mbar_wait(BAR(C::K_FULL + s1), (it / C::kSlots) & 1, abort_flag)) break;
+                ++it;
+                uint32_t s2 = s1;
+                if (!SHARED_K) {
+                    s2 = it % C::kSlots;
+                    if (!mbar_wait(BAR(C::K_FULL + s2), (it / C::kSlots) & 1, abort_flag)) break;
+                    ++it;
+                }
+                tc_fence_after();
+                for (int t = 0; t < ntiles; ++t) {
+                    if (j >= nkt[t]) continue;
+                    if (j > 0) {
+                        if (!mbar_wait(BAR(C::S_FREE + t), (j - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const uint32_t d1 = tmem + t * 256;
+                    const uint32_t d2 = d1 + 128;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+                        mma_bf16_ss(d1, sw128_desc(sb + C::kQ1 + t * C::kTile + off, 16, 1024),
+                                    sw128_desc(sb + C::kK + s1 * C::kTile + off, 16, 1024), idesc,
+                                    k > 0);
+                    }
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+                        mma_bf16_ss(d2, sw128_desc(sb + C::kQ2 + t * C::kTile + off, 16, 1024),
+                                    sw128_desc(sb + C::kK + s2 * C::kTile + off, 16, 1024), idesc,
+                                    k > 0);
+                    }
+                    mma_commit(BAR(C::S_FULL + t));
+                }
+                mma_commit(BAR(C::K_EMPTY + s1));
+                if (!SHARED_K) mma_commit(BAR(C::K_EMPTY + s2));
+            }
+            // drain: every MMA this thread issued must finish before TMEM is released
+            mma_commit(BAR(C::DONE));
+            drain_wait(BAR(C::DONE), 0);
+        }
+    } else if (warp >= 4) {
+        // ================================================================ statistics
+        const int t = (warp - 4) >> 2;
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        if (t < ntiles) {
+            const int i = q0[t] + r;
+            const uint32_t tS1 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(t * 256);
+            const uint32_t tS2 = tS1 + 128;
+            const float sl2 = p.sl2;
+            float m1 = -1e30f, l1 = 0.f, m2 = -1e30f, l2 = 0.f, acc = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nkt[t]; ++j) {
+                if (!mbar_wait(BAR(C::S_FULL + t), j & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int kb = j * 128;
+                const bool masked = (kb + 128 > p.NK) || (p.causal && kb + 127 > q0[t]);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t xa[32], ya[32];
+                    tmem_ld32(tS1 + c * 32, xa);
+                    tmem_ld32(tS2 + c * 32, ya);
+                    tmem_wait_ld();
+                    if (c == 3) {
+                        tc_fence_before();
+                        mbar_arrive(BAR(C::S_FREE + t));
+                    }
+                    if (!masked) {
+                        fold_chunk<false>(xa, ya, 0u, sl2, m1, l1, m2, l2, acc);
+                    } else {
+                        const int k0 = kb + c * 32;
+                        int lim = p.NK - k0;                       // keys k0 + k valid if k < lim
+                        if (p.causal) lim = min(lim, i - k0 + 1);  // ... and k0 + k <= i
+                        const uint32_t valid = lim >= 32 ? 0xFFFFFFFFu
+                                             : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+                        fold_chunk<true>(xa, ya, valid, sl2, m1, l1, m2, l2, acc);
+                    }
+                }
+            }
+            if (ok && i < p.NQ) {
+                const float LN2 = 0.6931471805599453f;
+                const float lg1 = log2f(l1);
+                const float lg2 = log2f(l2);
+                const size_t o = (size_t)bh * p.NQ + i;
+                p.lse1[o] = (m1 + lg1) * LN2;
+                p.lse2[o] = (m2 + lg2) * LN2;
+                p.kl[o] = p.scale * acc / l1 + ((m2 - m1) + (lg2 - lg1)) * LN2;
+            }
+        }
+    }
+
+    // ---- teardown: all TMEM readers and the MMA issuer are done past this barrier
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+#undef BAR
+}
+
+}  // namespace skl

@@ -1,0 +1,186 @@
+// streamkl.cu -- host side of libstreamkl: argument checks, TMA descriptors and launches
+// behind the C ABI declared in include/streamkl.h.  The whole library is this one
+// translation unit (the kernels are headers), so the device status word has one home.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "streamkl.h"
+#include "sm100.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+thread_local char t_last_cuda_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+    snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+    return STREAMKL_ERR_CUDA;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 3-D view [planes, rows, d] of a dense bf16 tensor, 128-row x 64-column boxes, 128-byte
+// swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* map, const void* base, long long planes, long long rows, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) {
+        snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
+        return STREAMKL_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)",
+                 (int)r);
+        return STREAMKL_ERR_CUDA;
+    }
+    return STREAMKL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || NQ < 1 || NK < 1 || d < 1) return STREAMKL_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return STREAMKL_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return STREAMKL_ERR_UNSUPPORTED;
+    if (Hq % Hkv != 0) return STREAMKL_ERR_UNSUPPORTED;
+    if (causal && NQ != NK) return STREAMKL_ERR_UNSUPPORTED;
+    if ((long long)B * Hq * NQ >= (1ll << 31) || (long long)B * Hkv * NK >= (1ll << 31))
+        return STREAMKL_ERR_UNSUPPORTED;
+    return STREAMKL_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    return STREAMKL_OK;
+}
+
+template <int D, bool SHARED>
+int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
+               const CUtensorMap& k2, const skl::FwdParams& p, int grid, cudaStream_t st) {
+    auto kern = skl::streamkl_fwd_kernel<D, SHARED>;
+    constexpr int smem = skl::FwdCfg<D>::kSmem;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    kern<<<grid, skl::kFwdThreads, smem, st>>>(q1, q2, k1, k2, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "streamkl_fwd launch");
+    return STREAMKL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int streamkl_version(void) { return 100; }
+
+const char* streamkl_status_string(int status) {
+    switch (status) {
+        case STREAMKL_OK: return "ok";
+        case STREAMKL_ERR_INVALID_ARG: return "invalid argument";
+        case STREAMKL_ERR_UNSUPPORTED: return "unsupported shape, scale or alignment";
+        case STREAMKL_ERR_CUDA: return "CUDA error";
+        case STREAMKL_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* streamkl_last_cuda_error(void) { return t_last_cuda_error; }
+
+int streamkl_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, skl::g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "read device status");
+    if (v != 0) {
+        e = cudaMemcpyToSymbol(skl::g_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+    }
+    return v;
+}
+
+int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
+                 int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                 float* kl, float* lse1, float* lse2, void* stream) {
+    if (!q1 || !k1 || !q2 || !k2 || !kl || !lse1 || !lse2) return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    if (!aligned16(q1) || !aligned16(k1) || !aligned16(q2) || !aligned16(k2) || !aligned16(kl) ||
+        !aligned16(lse1) || !aligned16(lse2))
+        return STREAMKL_ERR_UNSUPPORTED;
+    const bool shared = (k1 == k2);
+    CUtensorMap mq1, mq2, mk1, mk2;
+    if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d))) return rc;
+    if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d))) return rc;
+    if ((rc = make_map(&mk1, k1, (long long)B * Hkv, NK, d))) return rc;
+    if ((rc = make_map(&mk2, k2, (long long)B * Hkv, NK, d))) return rc;
+    skl::FwdParams p;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NQ = NQ; p.NK = NK;
+    p.causal = causal ? 1 : 0;
+    p.n_qblk = (NQ + 255) / 256;
+    p.sl2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.kl = kl; p.lse1 = lse1; p.lse2 = lse2;
+    const long long grid = (long long)B * Hq * p.n_qblk;
+    if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) {
+        return shared ? launch_fwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                      : launch_fwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+    }
+    return shared ? launch_fwd<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                  : launch_fwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+}
+
+size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d) {
+    if (B < 1 || Hq < 1 || NQ < 1 || (d != 64 && d != 128)) return 0;
+    return (size_t)B * Hq * NQ * d * sizeof(float);
+}
+
+int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
+                 const uint16_t* k2, const float* kl, const float* lse1, const float* lse2,
+                 const float* dkl, int B, int Hq, int Hkv, int NQ, int NK, int d, float scale,
+                 int causal, uint16_t* dq, uint16_t* dk, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    if (mode != 1 && mode != 2) return STREAMKL_ERR_INVALID_ARG;
+    if (!q1 || !k1 || !q2 || !k2 || !kl || !lse1 || !lse2 || !dkl || !dq || !dk || !workspace)
+        return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    if (workspace_bytes < streamkl_bwd_workspace_bytes(B, Hq, NQ, d)) return STREAMKL_ERR_INVALID_ARG;
+    const void* ptrs[] = {q1, k1, q2, k2, kl, lse1, lse2, dkl, dq, dk, workspace};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return STREAMKL_ERR_UNSUPPORTED;
+    (void)stream;
+    return STREAMKL_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+/*
+ * streamkl.h -- C ABI of libstreamkl, a B200 (sm_100a) fused attention KL divergence.
+ *
+ * The operation ("StreamKL: Fast and Memory-Efficient KL Divergence for Boosting Attention
+ * Distillation", abstract; StreamKL technical summary, gist.science, Portuguese,
+ * "Definição do Problema"): for batch b, query head h and query row i,
+ *
+ *     s_t[j] = scale * <Q_t[b,h,i,:], K_t[b,h/(Hq/Hkv),j,:]>,   t = 1, 2
+ *     P_t    = softmax of s_t over the valid keys (j < NK, and j <= i when causal)
+ *     KL_i   = sum_j P1[j] * (log P1[j] - log P2[j])
+ *
+ * computed without ever forming P1 or P2 in memory.  Grouped query heads follow the GQA
+ * definition of the KV-cache lecture notes (hackmd, "3. 架構層級的記憶體妥協").
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument is a DEVICE pointer owned by the caller; the library keeps no
+ *    reference after the call returns and allocates no device memory.
+ *  - Tensors are dense and row-major with the head dimension innermost:
+ *      Q1, Q2, dQ : bf16 [B, Hq, NQ, d]        K1, K2, dK : bf16 [B, Hkv, NK, d]
+ *      kl, lse1, lse2, dkl : fp32 [B, Hq, NQ]
+ *    bf16 is IEEE-754 binary32 truncated to its upper 16 bits (passed as uint16_t).
+ *  - Supported: d in {64, 128}; B, Hq, Hkv, NQ, NK >= 1; Hq % Hkv == 0; scale > 0 and
+ *    finite; causal requires NQ == NK (the mask is j <= i); every pointer 16-byte aligned;
+ *    B*Hq*NQ and B*Hkv*NK below 2^31 rows.  Anything else returns STREAMKL_ERR_UNSUPPORTED
+ *    (shape or alignment outside the supported set) or STREAMKL_ERR_INVALID_ARG (null
+ *    pointer, non-positive size, bad mode), and nothing is launched.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream).  A return of STREAMKL_OK means the work was enqueued.  Errors that happen on
+ *    the device later (a bounded pipeline wait that ran out) are recorded in a device status
+ *    word that streamkl_device_status() reads.  On any error the outputs are undefined.
+ *  - No call aborts the process or traps on the device.
+ *  - K1 == K2 (the same pointer) means one shared key tensor: it is read once per tile.
+ */
+#ifndef STREAMKL_H
+#define STREAMKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    STREAMKL_OK = 0,
+    STREAMKL_ERR_INVALID_ARG = 1,  /* null pointer, size < 1, mode not 1/2, workspace too small */
+    STREAMKL_ERR_UNSUPPORTED = 2,  /* d not 64/128, Hq % Hkv, causal with NQ != NK, alignment */
+    STREAMKL_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed (launch, memset) */
+    STREAMKL_ERR_TIMEOUT = 4       /* a kernel gave up on a pipeline wait (device status only) */
+};
+
+/*
+ * Forward.  One pass over the key tiles per query row, keeping five running scalars per
+ * row (m1, l1, m2, l2, acc) and returning KL = acc/l1 + LSE2 - LSE1 with
+ * LSE_t = m_t + log l_t (StreamKL technical summary, "1. Formulação Online (Passagem
+ * Forward)"; running sums rescaled by exp(m_old - m_new) when a maximum grows, as in the
+ * FlashAttention lecture notes, hackmd, "4. Flash Attention 的核心數學重構").  Causal key
+ * tiles past the diagonal are skipped entirely.
+ *
+ *   q1, k1, q2, k2 : bf16 inputs (see conventions); k1 == k2 selects the shared-key path.
+ *   kl, lse1, lse2 : fp32 [B,Hq,NQ] outputs, overwritten; natural-log units.  These three
+ *                    vectors are the whole saved state of the backward ("2. Estratégia de
+ *                    Recomputação", "Estado Salvo").
+ * Extra device memory: none.
+ */
+int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
+                 int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                 float* kl, float* lse1, float* lse2, void* stream);
+
+/*
+ * Bytes of fp32 workspace streamkl_bwd needs: B*Hq*NQ*d*4 (the dQ accumulator).  Returns
+ * 0 for sizes outside the supported range.
+ */
+size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d);
+
+/*
+ * Backward of sum_i dkl[i] * KL_i, recomputing P_t = exp(S_t - LSE_t) tile by tile from the
+ * saved LSEs (technical summary, "2. Estratégia de Recomputação (Passagem Backward)",
+ * "Regeneração").  With g = dkl:
+ *   mode 1 (P1 fixed, "Configuração 1"): dS2 = g * (P2 - P1); outputs dQ2, dK2.
+ *   mode 2 (P2 fixed, "Configuração 2"): dS1 = g * P1 * ((S1-LSE1) - (S2-LSE2) - KL),
+ *        with the log-ratio taken from logit differences and the saved LSEs, never from
+ *        log P ("Estabilidade Numérica"); outputs dQ1, dK1.
+ *   dQ_t = scale * dS_t K_t,  dK_t = scale * dS_t^T Q_t summed over the query heads that
+ *   share the KV head.  The fixed distribution gets no gradient; with k1 == k2 the
+ *   returned dk is the gradient through the free distribution only.
+ *
+ *   kl, lse1, lse2 : the forward's outputs for the same inputs (read only).
+ *   dkl            : fp32 [B,Hq,NQ] upstream gradient (read only).
+ *   dq             : bf16 [B,Hq,NQ,d] output, overwritten.
+ *   dk             : bf16 [B,Hkv,NK,d] output, overwritten.
+ *   workspace      : caller-owned device buffer of at least
+ *                    streamkl_bwd_workspace_bytes(B,Hq,NQ,d) bytes, 16-byte aligned; its
+ *                    contents on entry do not matter and are undefined on exit.  Two calls
+ *                    that run at the same time need two workspaces.
+ */
+int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
+                 const uint16_t* k2, const float* kl, const float* lse1, const float* lse2,
+                 const float* dkl, int B, int Hq, int Hkv, int NQ, int NK, int d, float scale,
+                 int causal, uint16_t* dq, uint16_t* dk, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Static text for a status code (never NULL). */
+const char* streamkl_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the current
+ * device.  Returns STREAMKL_OK, STREAMKL_ERR_TIMEOUT (a kernel abandoned a pipeline wait
+ * and left its outputs undefined) or STREAMKL_ERR_CUDA (the synchronisation itself failed;
+ * cudaGetLastError text is available through streamkl_last_cuda_error).
+ */
+int streamkl_device_status(void* stream);
+
+/* Text of the last CUDA error the library saw on this host thread ("" if none). */
+const char* streamkl_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int streamkl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMKL_H */

@@ -1,0 +1,117 @@
+"""The C-ABI library builds, loads without a GPU, exports every declared symbol, and rejects
+bad arguments on the host before touching the device (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_kl_divergence_02_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(streamkl_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"streamkl_fwd", "streamkl_bwd", "streamkl_bwd_workspace_bytes"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(binding.EXPORTS) == set(names)
+
+
+def test_status_strings_and_version(lib):
+    assert binding.version() >= 100
+    for code in range(5):
+        assert binding.status_string(code)
+    assert binding.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    assert binding.streamkl_bwd_workspace_bytes(1, 32, 16384, 128) == 32 * 16384 * 128 * 4
+    assert binding.streamkl_bwd_workspace_bytes(2, 3, 5, 64) == 2 * 3 * 5 * 64 * 4
+    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 96) == 0
+    assert binding.streamkl_bwd_workspace_bytes(0, 1, 1, 64) == 0
+
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced: every call below fails its checks first
+
+
+def fwd_call(**kw):
+    args = dict(q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, B=1, Hq=2, Hkv=1, NQ=8, NK=8, d=64,
+                scale=0.125, causal=0, kl=FAKE, lse1=FAKE, lse2=FAKE, stream=0)
+    args.update(kw)
+    return binding.streamkl_fwd(**args)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q1=None), binding.ERR_INVALID_ARG),
+    (dict(kl=None), binding.ERR_INVALID_ARG),
+    (dict(B=0), binding.ERR_INVALID_ARG),
+    (dict(NQ=-1), binding.ERR_INVALID_ARG),
+    (dict(d=96), binding.ERR_UNSUPPORTED),
+    (dict(d=256), binding.ERR_UNSUPPORTED),
+    (dict(Hq=3, Hkv=2), binding.ERR_UNSUPPORTED),
+    (dict(causal=1, NQ=8, NK=9), binding.ERR_UNSUPPORTED),
+    (dict(scale=0.0), binding.ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), binding.ERR_UNSUPPORTED),
+    (dict(scale=-1.0), binding.ERR_UNSUPPORTED),
+    (dict(q2=FAKE + 8), binding.ERR_UNSUPPORTED),
+    (dict(lse1=FAKE + 4), binding.ERR_UNSUPPORTED),
+    (dict(B=1 << 20, Hq=1 << 6, Hkv=1, NQ=1 << 6), binding.ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_on_host(lib, kw, want):
+    assert fwd_call(**kw) == want
+
+
+def bwd_call(**kw):
+    args = dict(mode=1, q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, kl=FAKE, lse1=FAKE, lse2=FAKE,
+                dkl=FAKE, B=1, Hq=2, Hkv=1, NQ=8, NK=8, d=64, scale=0.125, causal=0, dq=FAKE,
+                dk=FAKE, workspace=FAKE, workspace_bytes=2 * 8 * 64 * 4, stream=0)
+    args.update(kw)
+    return binding.streamkl_bwd(**args)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(mode=0), binding.ERR_INVALID_ARG),
+    (dict(mode=3), binding.ERR_INVALID_ARG),
+    (dict(dq=None), binding.ERR_INVALID_ARG),
+    (dict(workspace=None), binding.ERR_INVALID_ARG),
+    (dict(workspace_bytes=2 * 8 * 64 * 4 - 4), binding.ERR_INVALID_ARG),
+    (dict(d=32), binding.ERR_UNSUPPORTED),
+    (dict(causal=1, NK=7), binding.ERR_UNSUPPORTED),
+    (dict(dk=FAKE + 2), binding.ERR_UNSUPPORTED),
+    (dict(workspace=FAKE + 4), binding.ERR_UNSUPPORTED),
+])
+def test_bwd_rejects_on_host(lib, kw, want):
+    assert bwd_call(**kw) == want
+
+
+def test_header_is_plain_c():
+    """The public header compiles as C99 with no CUDA or torch headers."""
+    import subprocess
+    import tempfile
+    with tempfile.TemporaryDirectory() as td:
+        src = os.path.join(td, "t.c")
+        with open(src, "w") as f:
+            f.write('#include "streamkl.h"\n'
+                    'int (*volatile vfn)(void) = streamkl_version;\n'
+                    'int main(void){return vfn != streamkl_version;}\n')
+        subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I",
+                               os.path.join(ROOT, "include"), src, "-o", os.path.join(td, "t.o")])

@@ -1,0 +1,138 @@
+"""Forward parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_kl_divergence_02_b200 import binding, inputs
+
+from parity import check_fwd, host64, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+def both(w):
+    t = inputs.make(w, device="cuda")
+    got = run_fwd(t, w)
+    want = oracle.fwd(host64(t["q1"]), host64(t["k1"]), host64(t["q2"]), host64(t["k2"]),
+                      scale=w.scale, causal=w.causal)
+    return got, want, t
+
+
+def test_tiny_workload():
+    w = inputs.WORKLOADS["tiny"]
+    got, want, _ = both(w)
+    check_fwd(got, want, "tiny")
+
+
+CASES = [
+    # B, Hq, Hkv, NQ, NK, d, causal, shared
+    (1, 2, 2, 640, 640, 128, False, False),
+    (1, 2, 2, 640, 640, 128, True, False),
+    (1, 2, 2, 640, 640, 128, True, True),
+    (2, 4, 2, 300, 333, 64, False, False),     # GQA, ragged rows and keys
+    (1, 3, 1, 129, 129, 64, True, True),       # one row past a tile, causal
+    (1, 2, 2, 257, 257, 128, True, False),     # one row past a 256-row CTA block
+    (1, 1, 1, 1, 1, 128, False, True),         # single key, single row
+    (1, 1, 1, 1, 1000, 64, False, False),      # single row, ragged keys
+    (1, 2, 1, 200, 1, 64, False, False),       # single key
+    (1, 1, 1, 40, 40, 128, True, True),        # smaller than one tile
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dHq%dHkv%dNQ%dNK%dd%d%s%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "", "s" if c[7] else ""))
+def test_shapes(case):
+    B, Hq, Hkv, NQ, NK, d, causal, shared = case
+    w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=NQ + NK + d)
+    got, want, _ = both(w)
+    check_fwd(got, want, str(case))
+
+
+def test_peaked_and_flat_rows():
+    """Per-head scaled queries (the grouped-query recipe) at a reduced size: peaked rows
+    (large scale) and flat rows (small scale) in one call."""
+    w = inputs.custom(2, 8, 2, 384, 1000, 64, False, False, seed=11, head_scaled=True)
+    got, want, _ = both(w)
+    check_fwd(got, want, "peaked")
+
+
+def test_identical_inputs_give_zero_kl():
+    w = inputs.custom(1, 2, 2, 300, 300, 128, True, True, seed=3)
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q1"], t["k1"], scale=w.scale, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(l1, l2)
+    assert torch.all(kl == 0)
+
+
+def test_causal_row_zero_and_nonnegative():
+    w = inputs.custom(1, 4, 4, 512, 512, 128, True, False, seed=5)
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=True)
+    kl = kl.cpu()
+    assert torch.all(kl[:, :, 0].abs() <= 1e-6)
+    assert kl.min() >= -2e-3
+    s00 = (t["q1"][0, :, 0].float() * t["k1"][0, :, 0].float()).sum(-1) * w.scale
+    assert torch.allclose(l1[0, :, 0].cpu(), s00.cpu(), atol=1e-3)
+
+
+def test_deterministic():
+    w = inputs.custom(1, 4, 4, 512, 512, 128, True, True, seed=6)
+    t = inputs.make(w, device="cuda")
+    a = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=True)
+    b = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_non_default_scale_and_stream():
+    w = inputs.custom(1, 2, 2, 256, 384, 128, False, False, seed=8)
+    t = inputs.make(w, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        got = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=0.3, causal=False, stream=s)
+    s.synchronize()
+    want = oracle.fwd(host64(t["q1"]), host64(t["k1"]), host64(t["q2"]), host64(t["k2"]), scale=0.3)
+    check_fwd(tuple(x.cpu().double().numpy() for x in got), want, "scale0.3")
+
+
+def test_no_extra_device_memory():
+    """The forward allocates nothing: torch's allocator sees no growth and the free device
+    memory reported by the driver does not drop across the call."""
+    w = inputs.custom(1, 8, 8, 2048, 2048, 128, True, True, seed=9)
+    t = inputs.make(w, device="cuda")
+    out = tuple(torch.empty((1, 8, 2048), device="cuda") for _ in range(3))
+    binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], causal=True, out=out)  # warm
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], causal=True, out=out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 >= free0
+
+
+@pytest.mark.parametrize("name", ["b2h8n4k", "headline", "gqa"])
+def test_full_size_sampled(name):
+    """Full-size workloads in the launch configuration the benchmark times; the oracle
+    checks 64 seeded random rows per (batch, head)."""
+    base = inputs.WORKLOADS[name]
+    for causal in ((False, True) if name == "b2h8n4k" else (base.causal,)):
+        w = inputs.variant(base, causal=causal)
+        t = inputs.make(w, device="cuda")
+        kl, l1, l2 = run_fwd(t, w)
+        rng = np.random.default_rng(123)
+        rows = []
+        for bh in range(w.B * w.Hq):
+            rows += list(bh * w.NQ + rng.choice(w.NQ, size=64, replace=False))
+        rows += [0, w.NQ - 1, w.B * w.Hq * w.NQ - 1]
+        rows = np.array(sorted(set(rows)))
+        want = oracle.fwd_rows(host64(t["q1"]), host64(t["k1"]), host64(t["q2"]), host64(t["k2"]),
+                               rows, scale=w.scale, causal=w.causal)
+        got = tuple(x.reshape(-1)[rows] for x in (kl, l1, l2))
+        check_fwd(got, want, "%s causal=%s" % (name, causal))
+        assert np.all(kl >= -2e-3)
