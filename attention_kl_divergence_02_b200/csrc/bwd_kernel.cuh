@@ -1,0 +1,470 @@
+// bwd_kernel.cuh -- StreamKL backward on sm_100a.
+//
+// Gradient of sum_i g_i KL_i with one distribution held fixed (StreamKL technical summary,
+// gist.science, Portuguese, "2. Estratégia de Recomputação (Passagem Backward)"):
+//   mode 1 (P1 fixed):  dS2 = g * (P2 - P1)                         -> dQ2, dK2
+//   mode 2 (P2 fixed):  dS1 = g * P1 * ((S1-LSE1) - (S2-LSE2) - KL) -> dQ1, dK1
+// with P_t = exp(S_t - LSE_t) regenerated tile by tile from the saved LSEs ("Regeneração")
+// and the mode-2 log-ratio taken from logit differences, never log P ("Estabilidade
+// Numérica").  dQ = scale * dS K, dK = scale * dS^T Q.
+//
+// One CTA owns one 128-key tile of one (batch, KV head) and visits every 128-row query
+// tile of every query head in the KV group that can see it (causal: from the diagonal
+// on), so each (query tile, key tile) pair is visited exactly once ("Fusão de Kernel").
+// Per visit n:
+//   tensor core : S1^T = K1 Q1^T, S2^T = K2 Q2^T           (TMEM, lane = key)
+//   4 warpgroups: dS^T for 32 query columns each -> bf16, written once into a swizzled
+//                 shared tile that serves both MMAs below
+//   tensor core : dK += dS^T Q_free   (TMEM accumulator over all visits: no atomics)
+//                 dQp  = dS K_free    (TMEM, lane = query row)
+//   4 warpgroups: dQp added into the fp32 dQ workspace with vector atomics (the live rows
+//                 of the workspace stay resident in L2)
+// The MMA issuer looks one visit ahead: S of visit n+1 runs on the tensor core while the
+// warpgroups turn S of visit n into dS (needs two query stages in shared memory).
+//
+// Roles (640 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
+// warps 2-3 idle, warps 4..19 = four 128-thread compute warpgroups (warp w touches TMEM
+// lanes 32*(w%4)..+31).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace skl {
+
+struct BwdParams {
+    int B, Hq, Hkv, NQ, NK;
+    int causal;
+    int mode;
+    int nkt;        // key tiles per (b, KV head)
+    int nqt;        // query tiles per head
+    float sl2;      // scale * log2(e)
+    float scale;
+    const float* kl;
+    const float* lse1;
+    const float* lse2;
+    const float* dkl;
+    float* dq_ws;   // fp32 [B,Hq,NQ,d]
+    uint16_t* dk;   // bf16 [B,Hkv,NK,d]
+};
+
+constexpr int kBwdThreads = 640;
+constexpr int kBwdWG = 4;   // compute warpgroups
+
+template <int D, bool SHARED_K>
+struct BwdCfg {
+    static constexpr int kTile = 128 * D * 2;
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kBox = 128 * 128;
+    static constexpr int kQS = (D == 128 && !SHARED_K) ? 1 : 2;   // query stages
+    static constexpr int kNK = SHARED_K ? 1 : 2;                   // resident key tiles
+    static constexpr int kK = 0;                                   // key tile i at kK + i*kTile
+    static constexpr int kQ = kNK * kTile;                         // stage s: Q1 at kQ + s*2*kTile, Q2 after
+    static constexpr int kDS = kQ + kQS * 2 * kTile;               // dS^T tile, 128 x 128 bf16
+    static constexpr int kCst = kDS + 128 * 128 * 2;               // per-query constants [16 warps][32] float4
+    static constexpr int kBar = kCst + 4 * kBwdWG * 32 * 16;
+    static constexpr int K_FULL = 0;
+    static constexpr int Q_FULL = 1;                // + s
+    static constexpr int Q_EMPTY = 1 + kQS;         // + s
+    static constexpr int S_FULL = 1 + 2 * kQS;
+    static constexpr int S_FREE = S_FULL + 1;
+    static constexpr int DS_FULL = S_FULL + 2;
+    static constexpr int DS_FREE = S_FULL + 3;
+    static constexpr int DQ_FULL = S_FULL + 4;
+    static constexpr int DQ_FREE = S_FULL + 5;
+    static constexpr int DK_FULL = S_FULL + 6;
+    static constexpr int DONE = S_FULL + 7;
+    static constexpr int kNumBars = DONE + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kSmem = kMisc + 16 + 1024;
+    static constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDK = 256, kColDQ = 384;
+};
+
+// Visit n of a CTA -> (query head, query tile).  Causal: every head of the group, query
+// tiles from the diagonal on.  Non-causal: all (head, tile) pairs, rotated by the key tile
+// index so that CTAs of one head start on different dQ rows.
+struct BwdSchedule {
+    int hk0, G, nqt, kt, causal, count;
+    __device__ BwdSchedule(const BwdParams& p, int hk, int kt_) {
+        G = p.Hq / p.Hkv;
+        hk0 = hk * G;
+        nqt = p.nqt;
+        kt = kt_;
+        causal = p.causal;
+        count = causal ? G * (nqt - kt) : G * nqt;
+    }
+    __device__ void visit(int n, int& h, int& qt) const {
+        if (causal) {
+            const int per = nqt - kt;
+            h = hk0 + n / per;
+            qt = kt + n % per;
+        } else {
+            const int u = (n + kt) % count;
+            h = hk0 + u / nqt;
+            qt = u % nqt;
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 16 consecutive fp32 TMEM columns of the thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// D/4 columns of one TMEM lane (32 for d = 128, 16 for d = 64).
+template <int D>
+__device__ __forceinline__ void tmem_ld_quarter(uint32_t taddr, float (&v)[D / 4]) {
+    if constexpr (D == 128) {
+        uint32_t r[32];
+        tmem_ld32(taddr, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+    } else {
+        uint32_t r[16];
+        tmem_ld16(taddr, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+    }
+}
+
+template <int D, bool SHARED_K>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
+                    const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
+                    const BwdParams p) {
+    using C = BwdCfg<D, SHARED_K>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(smem);
+    const uint32_t bar0 = sb + C::kBar;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+#define BAR(i) (bar0 + 8u * (uint32_t)(i))
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int BHk = p.B * p.Hkv;
+    const int kt = blockIdx.x / BHk;     // key tile; kt = 0 (most visits when causal) first
+    const int bhk = blockIdx.x % BHk;
+    const int b = bhk / p.Hkv;
+    const int hk = bhk % p.Hkv;
+    const int k0 = kt * 128;
+    const BwdSchedule sched(p, hk, kt);
+    const int N = sched.count;
+    const bool mode1 = (p.mode == 1);
+    // the free distribution's operands: mode 1 -> (Q2, K2), mode 2 -> (Q1, K1)
+    const uint32_t kfree = sb + C::kK + ((SHARED_K || !mode1) ? 0 : C::kTile);
+    const uint32_t k2tile = sb + C::kK + (SHARED_K ? 0 : C::kTile);
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(C::K_FULL), 1);
+        for (int s = 0; s < C::kQS; ++s) {
+            mbar_init(BAR(C::Q_FULL + s), 1);
+            mbar_init(BAR(C::Q_EMPTY + s), 1);
+        }
+        mbar_init(BAR(C::S_FULL), 1);
+        mbar_init(BAR(C::S_FREE), 32 * 4 * kBwdWG);
+        mbar_init(BAR(C::DS_FULL), 32 * 4 * kBwdWG);
+        mbar_init(BAR(C::DS_FREE), 1);
+        mbar_init(BAR(C::DQ_FULL), 1);
+        mbar_init(BAR(C::DQ_FREE), 32 * 4 * kBwdWG);
+        mbar_init(BAR(C::DK_FULL), 1);
+        mbar_init(BAR(C::DONE), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ1);
+            tma_prefetch_desc(&tmQ2);
+            tma_prefetch_desc(&tmK1);
+            if (!SHARED_K) tma_prefetch_desc(&tmK2);
+            mbar_arrive_expect_tx(BAR(C::K_FULL), C::kNK * C::kTile);
+            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                tma_load_3d(sb + C::kK + bx * C::kBox, &tmK1, BAR(C::K_FULL), bx * 64, k0, bhk);
+                if (!SHARED_K)
+                    tma_load_3d(sb + C::kK + C::kTile + bx * C::kBox, &tmK2, BAR(C::K_FULL), bx * 64,
+                                k0, bhk);
+            }
+            int n = 0;
+            for (; n < N; ++n) {
+                const int s = n % C::kQS;
+                const int u = n / C::kQS;
+                if (u > 0 && !mbar_wait(BAR(C::Q_EMPTY + s), (u - 1) & 1, abort_flag)) break;
+                int h, qt;
+                sched.visit(n, h, qt);
+                const int bh = b * p.Hq + h;
+                const uint32_t q1s = sb + C::kQ + s * 2 * C::kTile;
+                const uint32_t q2s = q1s + C::kTile;
+                mbar_arrive_expect_tx(BAR(C::Q_FULL + s), 2 * C::kTile);
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_3d(q1s + bx * C::kBox, &tmQ1, BAR(C::Q_FULL + s), bx * 64, qt * 128, bh);
+                    tma_load_3d(q2s + bx * C::kBox, &tmQ2, BAR(C::Q_FULL + s), bx * 64, qt * 128, bh);
+                }
+            }
+            // drain every copy started here
+            drain_wait(BAR(C::K_FULL), 0);
+            for (int s = 0; s < C::kQS; ++s) {
+                if (n > s) {
+                    const int fills = (n - s - 1) / C::kQS + 1;
+                    drain_wait(BAR(C::Q_FULL + s), (fills - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // K-major A and B
+            constexpr uint32_t idK = idesc_bf16(128, D, 0, 1);     // dS^T K-major, Q MN-major
+            constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dS MN-major, K MN-major
+            auto issue_S = [&](int n) {
+                const int s = n % C::kQS;
+                const uint32_t q1s = sb + C::kQ + s * 2 * C::kTile;
+                const uint32_t q2s = q1s + C::kTile;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(sb + C::kK + off, 16, 1024),
+                                sw128_desc(q1s + off, 16, 1024), idS, k > 0);
+                }
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
+                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(k2tile + off, 16, 1024),
+                                sw128_desc(q2s + off, 16, 1024), idS, k > 0);
+                }
+                mma_commit(BAR(C::S_FULL));
+            };
+            auto issue_dK = [&](int n) {
+                const int s = n % C::kQS;
+                const uint32_t qf = sb + C::kQ + s * 2 * C::kTile + (mode1 ? C::kTile : 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
+                    mma_bf16_ss(tmem + C::kColDK,
+                                sw128_desc(sb + C::kDS + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
+                                sw128_desc(qf + k * 2048, C::kBox, 1024), idK, (n > 0 || k > 0));
+                }
+            };
+            auto issue_dQ = [&]() {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
+                    mma_bf16_ss(tmem + C::kColDQ, sw128_desc(sb + C::kDS + k * 2048, C::kBox, 1024),
+                                sw128_desc(kfree + k * 2048, C::kBox, 1024), idQ, k > 0);
+                }
+            };
+            bool ok = mbar_wait(BAR(C::K_FULL), 0, abort_flag);
+            if (ok && C::kQS >= 2) {
+                ok = mbar_wait(BAR(C::Q_FULL + 0), 0, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    issue_S(0);
+                }
+            }
+            for (int n = 0; n < N && ok; ++n) {
+                if (C::kQS >= 2) {
+                    if (n + 1 < N) {
+                        const int s1 = (n + 1) % C::kQS;
+                        if (!mbar_wait(BAR(C::Q_FULL + s1), ((n + 1) / C::kQS) & 1, abort_flag)) break;
+                        if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+                        tc_fence_after();
+                        issue_S(n + 1);
+                    }
+                } else {
+                    if (!mbar_wait(BAR(C::Q_FULL + 0), n & 1, abort_flag)) break;
+                    if (n > 0 && !mbar_wait(BAR(C::S_FREE), (n - 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    issue_S(n);
+                }
+                if (!mbar_wait(BAR(C::DS_FULL), n & 1, abort_flag)) break;
+                tc_fence_after();
+                issue_dK(n);
+                if (n > 0) {
+                    if (!mbar_wait(BAR(C::DQ_FREE), (n - 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                }
+                issue_dQ();
+                mma_commit(BAR(C::DS_FREE));
+                mma_commit(BAR(C::Q_EMPTY + n % C::kQS));
+                mma_commit(BAR(C::DQ_FULL));
+            }
+            mma_commit(BAR(C::DK_FULL));
+            mma_commit(BAR(C::DONE));
+            drain_wait(BAR(C::DONE), 0);
+        }
+    } else if (warp >= 4) {
+        // ================================================================ compute warpgroups
+        const int wg = (warp - 4) >> 2;         // query columns [32*wg, 32*wg + 32)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;      // TMEM lane: key row (S, dK) or query row (dQ)
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float sl2 = p.sl2;
+        const float scale = p.scale;
+        const float LOG2E = 1.4426950408889634f;
+        float4* cst = reinterpret_cast<float4*>(smem + C::kCst);
+        uint8_t* ds_tile = smem + C::kDS;
+        // this thread's 64 bytes of the dS^T row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
+        uint8_t* ds_row = ds_tile + (wg >> 1) * C::kBox + r * 128;
+        bool ok = true;
+        int prev_bh = 0, prev_q0 = 0;
+        auto drain_dq = [&](int n_done, int bh_, int q0_) -> bool {
+            if (!mbar_wait(BAR(C::DQ_FULL), n_done & 1, abort_flag)) return false;
+            tc_fence_after();
+            float v[D / 4];
+            tmem_ld_quarter<D>(lane_base + C::kColDQ + wg * (D / 4), v);
+            const int q = q0_ + r;
+            if (q < p.NQ) {
+                float4* dst = reinterpret_cast<float4*>(p.dq_ws + ((size_t)bh_ * p.NQ + q) * D + wg * (D / 4));
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k)
+                    atomicAdd(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+            }
+            return true;
+        };
+        for (int n = 0; n < N; ++n) {
+            int h, qt;
+            sched.visit(n, h, qt);
+            const int bh = b * p.Hq + h;
+            const int q0 = qt * 128;
+            // per-query constants of this warpgroup's 32 columns, one copy per warp (only
+            // warp-level syncs: no barrier that an aborting sibling warp could leave hanging)
+            float4* cbuf = cst + (warp - 4) * 32;
+            {
+                const int q = q0 + wg * 32 + lane;
+                float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (q < p.NQ) {
+                    const size_t o = (size_t)bh * p.NQ + q;
+                    const float L1 = p.lse1[o], L2 = p.lse2[o];
+                    c.x = L1 * LOG2E;
+                    c.y = L2 * LOG2E;
+                    c.z = p.dkl[o];
+                    c.w = mode1 ? 0.f : (L2 - L1 - p.kl[o]);
+                }
+                __syncwarp();          // the previous visit's reads of cbuf are done
+                cbuf[lane] = c;
+                __syncwarp();
+            }
+            if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t xa[32], ya[32];
+            tmem_ld32(lane_base + C::kColS1 + wg * 32, xa);
+            tmem_ld32(lane_base + C::kColS2 + wg * 32, ya);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(BAR(C::S_FREE));
+            // dS^T[r, q] for the 32 query columns
+            const bool diag = p.causal && (qt == kt);
+            const bool key_ok = (k0 + r < p.NK);   // zero-filled key rows past NK get dS = 0
+            const int qoff = wg * 32;      // column offset within the query tile
+            uint32_t packed[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                float ds[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float4 c = cbuf[k + e];
+                    const float x = __uint_as_float(xa[k + e]);
+                    const float y = __uint_as_float(ya[k + e]);
+                    const float p1 = ex2(fmaf(x, sl2, -c.x));
+                    float v;
+                    if (mode1) {
+                        const float p2 = ex2(fmaf(y, sl2, -c.y));
+                        v = c.z * (p2 - p1);
+                    } else {
+                        v = c.z * p1 * fmaf(scale, x - y, c.w);
+                    }
+                    if ((diag && r > qoff + k + e) || !key_ok) v = 0.f;
+                    ds[e] = v;
+                }
+                packed[k >> 1] = pack_bf16(ds[0], ds[1]);
+            }
+            if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const int cbase = (wg & 1) * 4;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int phys = (cbase + c) ^ (r & 7);
+                *reinterpret_cast<uint4*>(ds_row + phys * 16) =
+                    make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+            }
+            fence_async_smem();
+            mbar_arrive(BAR(C::DS_FULL));
+            if (n > 0) {
+                if (!drain_dq(n - 1, prev_bh, prev_q0)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_before();
+                mbar_arrive(BAR(C::DQ_FREE));
+            }
+            prev_bh = bh;
+            prev_q0 = q0;
+        }
+        if (ok && N > 0) ok = drain_dq(N - 1, prev_bh, prev_q0);
+        if (ok && mbar_wait(BAR(C::DK_FULL), 0, abort_flag)) {
+            tc_fence_after();
+            float v[D / 4];
+            tmem_ld_quarter<D>(lane_base + C::kColDK + wg * (D / 4), v);
+            if (k0 + r < p.NK) {
+                uint4* dst = reinterpret_cast<uint4*>(p.dk + ((size_t)bhk * p.NK + k0 + r) * D + wg * (D / 4));
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k)
+                    dst[k] = make_uint4(pack_bf16(v[8 * k] * scale, v[8 * k + 1] * scale),
+                                        pack_bf16(v[8 * k + 2] * scale, v[8 * k + 3] * scale),
+                                        pack_bf16(v[8 * k + 4] * scale, v[8 * k + 5] * scale),
+                                        pack_bf16(v[8 * k + 6] * scale, v[8 * k + 7] * scale));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+#undef BAR
+}
+
+// dq[i] = bf16(ws[i] * scale), eight elements per thread per step.
+__global__ void __launch_bounds__(256)
+streamkl_dq_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dq, size_t n8, float scale) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4*>(ws)[2 * i];
+        const float4 c = reinterpret_cast<const float4*>(ws)[2 * i + 1];
+        reinterpret_cast<uint4*>(dq)[i] =
+            make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
+                       pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+    }
+}
+
+}  // namespace skl

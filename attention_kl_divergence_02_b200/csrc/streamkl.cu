@@ -11,6 +11,7 @@
 #include "streamkl.h"
 #include "sm100.cuh"
 #include "fwd_kernel.cuh"
+#include "bwd_kernel.cuh"
 
 namespace {
 
@@ -92,6 +93,28 @@ int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
     kern<<<grid, skl::kFwdThreads, smem, st>>>(q1, q2, k1, k2, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_fwd launch");
+    return STREAMKL_OK;
+}
+
+template <int D, bool SHARED>
+int launch_bwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
+               const CUtensorMap& k2, const skl::BwdParams& p, int grid, size_t ws_bytes,
+               uint16_t* dq, cudaStream_t st) {
+    auto kern = skl::streamkl_bwd_kernel<D, SHARED>;
+    constexpr int smem = skl::BwdCfg<D, SHARED>::kSmem;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    cudaError_t e = cudaMemsetAsync(p.dq_ws, 0, ws_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace memset");
+    kern<<<grid, skl::kBwdThreads, smem, st>>>(q1, q2, k1, k2, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "streamkl_bwd launch");
+    const size_t n8 = ws_bytes / sizeof(float) / 8;
+    size_t blocks = (n8 + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    skl::streamkl_dq_convert_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.dq_ws, dq, n8, p.scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dq convert launch");
     return STREAMKL_OK;
 }
 
@@ -179,8 +202,33 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
     const void* ptrs[] = {q1, k1, q2, k2, kl, lse1, lse2, dkl, dq, dk, workspace};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return STREAMKL_ERR_UNSUPPORTED;
-    (void)stream;
-    return STREAMKL_ERR_UNSUPPORTED;
+    const bool shared = (k1 == k2);
+    CUtensorMap mq1, mq2, mk1, mk2;
+    if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d))) return rc;
+    if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d))) return rc;
+    if ((rc = make_map(&mk1, k1, (long long)B * Hkv, NK, d))) return rc;
+    if ((rc = make_map(&mk2, k2, (long long)B * Hkv, NK, d))) return rc;
+    skl::BwdParams p;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NQ = NQ; p.NK = NK;
+    p.causal = causal ? 1 : 0;
+    p.mode = mode;
+    p.nkt = (NK + 127) / 128;
+    p.nqt = (NQ + 127) / 128;
+    p.sl2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.kl = kl; p.lse1 = lse1; p.lse2 = lse2; p.dkl = dkl;
+    p.dq_ws = static_cast<float*>(workspace);
+    p.dk = dk;
+    const long long grid = (long long)B * Hkv * p.nkt;
+    if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
+    const size_t ws = streamkl_bwd_workspace_bytes(B, Hq, NQ, d);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) {
+        return shared ? launch_bwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st)
+                      : launch_bwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st);
+    }
+    return shared ? launch_bwd<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st)
+                  : launch_bwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st);
 }
 
 }  // extern "C"

@@ -1,0 +1,421 @@
+"""StreamKL benchmark: one step = the whole hot path on one batch of synthetic input:
+forward (KL, LSE1, LSE2) + backward with P1 fixed (dQ2, dK2) + backward with P2 fixed
+(dQ1, dK1), on the headline workload B=1, H=32, NQ=NK=16384, d=128, causal, shared keys,
+bf16 inputs (Q1 ~ N(0,1), Q2 = 0.8 Q1 + 0.6 N(0,1), K ~ N(0,1), seeded).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  value = whole-job TFLOP/s over all ranks, with FLOPs counted
+as 4d per unmasked (row, key) pair for the forward and 8d for each backward, causal pairs
+halved.  With N > 1 (torchrun, one process per GPU) every rank runs its own batch of the
+same workload (weak scaling, no data-path collective); timing is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a bounded
+sample of rows per step, rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd/bwd TFLOP/s & ms, H=32 N=16K d=128 causal bf16; % of B200 dense peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "headline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+L2_BYTES = 126 * 2**20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, power = [], None, set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    clk, mx = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                smax = mx
+                try:
+                    power.append(float(parts[3]))
+                except ValueError:
+                    pass
+                sm.append(clk)
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        loaded = [c for c in sm if smax and c > 0.3 * smax] or sm
+        loaded.sort()
+        med = loaded[len(loaded) // 2] if loaded else None
+        return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+def oracle_sample(w, n_rows, seed=0):
+    """Bounded oracle sample of one step: forward + both backward settings for ``n_rows``
+    random query rows of the workload (each row against all of its valid keys).  Returns
+    (seconds, flops) with FLOPs of the oracle's own work: 4d per pair for the forward and
+    6d per pair per backward row (recompute 4d + dQ 2d; the dK share of those rows is not
+    formed)."""
+    import numpy as np
+    import oracle
+    from attention_kl_divergence_02_b200 import inputs
+
+    t = _host_inputs(w)
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.B * w.Hq * w.NQ, size=n_rows, replace=False))
+    i = rows % w.NQ
+    pairs = float(np.sum(np.minimum(i + 1, w.NK) if w.causal else np.full(n_rows, w.NK)))
+    t0 = time.perf_counter()
+    oracle.fwd_rows(t["q1"], t["k1"], t["q2"], t["k2"], rows, scale=w.scale, causal=w.causal)
+    for mode in (1, 2):
+        oracle.bwd_dq_rows(mode, t["q1"], t["k1"], t["q2"], t["k2"], t["dkl"], rows,
+                           scale=w.scale, causal=w.causal)
+    dt = time.perf_counter() - t0
+    return dt, pairs * w.d * (4 + 6 + 6)
+
+
+_HOST = {}
+
+
+def _host_inputs(w):
+    from attention_kl_divergence_02_b200 import inputs
+    if w.name not in _HOST:
+        t = inputs.make(w, device="cpu")
+        _HOST[w.name] = {k: inputs.to_f64(v) for k, v in t.items()}
+    return _HOST[w.name]
+
+
+def cpu_baseline(w, target_s=15.0):
+    """Time the oracle on ~target_s seconds of sampled rows; TFLOP/s of that sample."""
+    import oracle
+    oracle.build()
+    cores = oracle.num_threads()
+    _host_inputs(w)
+    probe_rows = max(8, 2 * cores)
+    dt, _ = oracle_sample(w, probe_rows, seed=1)
+    n = int(min(w.B * w.Hq * w.NQ, max(probe_rows, probe_rows * target_s / max(dt, 1e-3))))
+    dt, flops = oracle_sample(w, n, seed=2)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "%d random query rows of the %s workload (all their valid keys): forward "
+                      "+ both backward settings (dQ rows) in the fp64 C oracle, OpenMP over rows; "
+                      "%.1f s" % (n, w.name, dt)}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from attention_kl_divergence_02_b200 import inputs
+    import oracle
+    oracle.build()
+    w = inputs.WORKLOADS[WORKLOAD]
+    cores = oracle.num_threads()
+    _host_inputs(w)
+    # size the per-step sample so that warmup + steps take about two minutes
+    dt, _ = oracle_sample(w, max(8, 2 * cores), seed=99)
+    per_row = dt / max(8, 2 * cores)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = max(cores, int(budget / max(per_row, 1e-6)))
+    for s in range(args.warmup):
+        oracle_sample(w, n, seed=1000 + s)
+    times, flops = [], 0.0
+    for s in range(args.steps):
+        dts, f = oracle_sample(w, n, seed=s)
+        times.append(dts)
+        flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "B1 H32 NQ=NK=16384 d128 causal shared-K (headline)",
+                   "sample_rows_per_step": n, "global_batch": 1, "seq_len": w.NQ},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "%d random query rows per step: forward + both backward "
+                                   "settings (dQ rows), fp64 C oracle" % n},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from attention_kl_divergence_02_b200 import binding, inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load()
+    base = inputs.WORKLOADS[WORKLOAD]
+    w = inputs.variant(base, seed=base.seed + 1000 * rank)  # own batch per rank
+    t = inputs.make(w, device=dev)
+    B, Hq, NQ, d = w.B, w.Hq, w.NQ, w.d
+    stream = torch.cuda.current_stream()
+    kl, l1, l2 = (torch.empty((B, Hq, NQ), device=dev) for _ in range(3))
+    g = {m: (torch.empty_like(t["q1"]), torch.empty_like(t["k1"])) for m in (1, 2)}
+    ws = torch.empty(binding.streamkl_bwd_workspace_bytes(B, Hq, NQ, d) // 4, device=dev)
+
+    def fwd():
+        binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal,
+                    out=(kl, l1, l2), stream=stream)
+
+    def bwd(mode):
+        binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], scale=w.scale,
+                    causal=w.causal, out=g[mode], workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        fwd(); bwd(1); bwd(2)
+    torch.cuda.synchronize()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
+
+    # ---- timed region: K steps, events between the three calls of every step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        fwd()
+        ev[k][1].record(stream)
+        bwd(1)
+        ev[k][2].record(stream)
+        bwd(2)
+        ev[k][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
+    total_ms = t_start.elapsed_time(t_end)
+    f_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    b1_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    b2_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    if world > 1:
+        x = torch.tensor([total_ms, f_ms, b1_ms, b2_ms], device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        total_ms, f_ms, b1_ms, b2_ms = x.tolist()
+    ms_step = total_ms / args.steps
+    step_flops = w.fwd_flops() + 2 * w.bwd_flops()
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.skip_e2e:
+        hin = {k: v.cpu().pin_memory() for k, v in inputs.make(w, device="cpu").items()}
+        dq_in = {k: torch.empty_like(v, device=dev) for k, v in hin.items() if k != "k2"}
+        hout = {"kl": torch.empty((B, Hq, NQ), pin_memory=True),
+                "lse1": torch.empty((B, Hq, NQ), pin_memory=True),
+                "lse2": torch.empty((B, Hq, NQ), pin_memory=True)}
+        for m in (1, 2):
+            hout["dq%d" % m] = torch.empty(tuple(t["q1"].shape), dtype=torch.bfloat16, pin_memory=True)
+            hout["dk%d" % m] = torch.empty(tuple(t["k1"].shape), dtype=torch.bfloat16, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for k, v in hin.items() if k != "k2")
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+
+        def e2e_step():
+            for k, v in dq_in.items():
+                v.copy_(hin[k], non_blocking=True)
+            k2 = dq_in["k1"]
+            binding.fwd(dq_in["q1"], dq_in["k1"], dq_in["q2"], k2, scale=w.scale, causal=w.causal,
+                        out=(kl, l1, l2), stream=stream)
+            for m in (1, 2):
+                binding.bwd(m, dq_in["q1"], dq_in["k1"], dq_in["q2"], k2, kl, l1, l2, dq_in["dkl"],
+                            scale=w.scale, causal=w.causal, out=g[m], workspace=ws, stream=stream)
+            hout["kl"].copy_(kl, non_blocking=True)
+            hout["lse1"].copy_(l1, non_blocking=True)
+            hout["lse2"].copy_(l2, non_blocking=True)
+            for m in (1, 2):
+                hout["dq%d" % m].copy_(g[m][0], non_blocking=True)
+                hout["dk%d" % m].copy_(g[m][1], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ne = max(3, min(args.steps, 10))
+        barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / ne
+        if world > 1:
+            x = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(x, op=dist.ReduceOp.MAX)
+            e_ms = x.item()
+        e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    calls = {"fwd": (f_ms, w.fwd_flops()), "bwd_mode1": (b1_ms, w.bwd_flops()),
+             "bwd_mode2": (b2_ms, w.bwd_flops())}
+    dom = max(calls, key=lambda k: calls[k][0])
+    dom_ms, dom_flops = calls[dom]
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    traffic = load_traffic(dom)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "B1 H32 NQ=NK=16384 d128 causal shared-K (headline); step = "
+                               "forward + backward P1-fixed + backward P2-fixed",
+                   "global_batch": world * B, "seq_len": NQ, "heads": Hq, "head_dim": d,
+                   "parallelism": "dp%d (independent batch per GPU, no collective)" % world,
+                   "l2": "inputs (3 x 128 MiB bf16) larger than the 126 MB L2; no flush"},
+        "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / (f_ms * 1e-3) / 1e12,
+        "bwd_mode1_ms": b1_ms, "bwd_mode1_tflops": w.bwd_flops() / (b1_ms * 1e-3) / 1e12,
+        "bwd_mode2_ms": b2_ms, "bwd_mode2_tflops": w.bwd_flops() / (b2_ms * 1e-3) / 1e12,
+        "pct_of_peak": {"fwd": 100 * w.fwd_flops() / (f_ms * 1e-3) / 1e12 / peak,
+                        "bwd_mode1": 100 * w.bwd_flops() / (b1_ms * 1e-3) / 1e12 / peak,
+                        "bwd_mode2": 100 * w.bwd_flops() / (b2_ms * 1e-3) / 1e12 / peak,
+                        "step": 100 * value / world / peak,
+                        "basis": "%s bf16 %.1f TFLOP/s (burst); nominal dense %.0f gives fwd %.1f%%"
+                                 % (peak_src, peak, NOMINAL_BF16_TFLOPS,
+                                    100 * w.fwd_flops() / (f_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS)},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": "%s bf16_tflops (burst)" % peak_src,
+                     "note": "achieved = algorithmic FLOPs per call / CUDA-event duration of the "
+                             "call on its stream%s" % (
+                                 "; the backward call also runs the dQ-workspace memset and the "
+                                 "dQ convert kernel" if dom.startswith("bwd") else "")},
+        "clocks": clk,
+        "gpu_launches": 5 * args.steps,
+        "e2e": e2e,
+    }
+    if world == 1 and rank == 0 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline(base)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get(kernel)
+    except (OSError, ValueError):
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU-oracle baseline leg")
+    ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

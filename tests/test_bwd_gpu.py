@@ -1,0 +1,154 @@
+"""Backward parity (both settings): the CUDA path through the C ABI against the fp64 oracle.
+Relative L2 error of dQ and dK per (batch, head) slice <= 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_kl_divergence_02_b200 import binding, inputs
+
+from parity import GRAD_TOL, check_grad, host64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_bwd(t, w, mode, workspace=None):
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal)
+    dq, dk = binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"],
+                         scale=w.scale, causal=w.causal, workspace=workspace)
+    assert binding.streamkl_device_status() == binding.OK
+    return dq.cpu().double().numpy(), dk.cpu().double().numpy()
+
+
+def host(t):
+    return {k: host64(v) for k, v in t.items()}
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_tiny_workload(mode):
+    w = inputs.WORKLOADS["tiny"]
+    t = inputs.make(w, device="cuda")
+    dq, dk = gpu_bwd(t, w, mode)
+    h = host(t)
+    odq, odk = oracle.bwd(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], scale=w.scale,
+                          causal=w.causal)
+    check_grad(dq, odq, "tiny dQ mode %d" % mode)
+    check_grad(dk, odk, "tiny dK mode %d" % mode)
+
+
+CASES = [
+    # B, Hq, Hkv, NQ, NK, d, causal, shared
+    (1, 2, 2, 640, 640, 128, False, False),
+    (1, 2, 2, 640, 640, 128, True, False),
+    (1, 2, 2, 640, 640, 128, True, True),
+    (2, 4, 2, 300, 333, 64, False, False),     # GQA, ragged rows and keys
+    (1, 4, 1, 200, 520, 64, False, True),      # GQA 4:1, shared keys
+    (1, 3, 1, 129, 129, 64, True, True),
+    (1, 2, 2, 257, 257, 128, True, False),
+    (1, 1, 1, 1, 1, 128, False, True),
+    (1, 1, 1, 40, 40, 128, True, True),
+    (1, 2, 1, 3, 700, 128, False, False),
+]
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dHq%dHkv%dNQ%dNK%dd%d%s%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "", "s" if c[7] else ""))
+def test_shapes(case, mode):
+    B, Hq, Hkv, NQ, NK, d, causal, shared = case
+    w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=NQ * 7 + NK + d)
+    t = inputs.make(w, device="cuda")
+    # non-uniform upstream gradient
+    t["dkl"] = torch.rand(t["dkl"].shape, generator=torch.Generator().manual_seed(1)).cuda() + 0.5
+    dq, dk = gpu_bwd(t, w, mode)
+    h = host(t)
+    odq, odk = oracle.bwd(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], scale=w.scale,
+                          causal=w.causal)
+    # natural size of a gradient entry is scale * g * |q| * |k|; fp32 rounding of the saved
+    # statistics leaves noise around 1e-7 of that where the exact gradient is zero
+    zero_atol = 1e-6 * w.scale * float(h["dkl"].max()) * max(np.abs(h["q1"]).max(), np.abs(h["q2"]).max()) \
+        * max(np.abs(h["k1"]).max(), np.abs(h["k2"]).max())
+    check_grad(dq, odq, "%s dQ mode %d" % (case, mode), zero_atol)
+    check_grad(dk, odk, "%s dK mode %d" % (case, mode), zero_atol)
+
+
+def test_workspace_contents_do_not_matter():
+    w = inputs.custom(1, 2, 2, 384, 384, 128, True, True, seed=4)
+    t = inputs.make(w, device="cuda")
+    n = binding.streamkl_bwd_workspace_bytes(1, 2, 384, 128) // 4
+    ws = torch.full((n,), float("nan"), device="cuda")
+    a = gpu_bwd(t, w, 1, workspace=ws)
+    ws.fill_(1e30)
+    b = gpu_bwd(t, w, 1, workspace=ws)
+    for x, y in zip(a, b):
+        assert np.all(np.isfinite(x))
+        assert rel_l2(x, y, axes=(2, 3)).max() < 1e-3
+
+
+def test_identical_distributions_give_zero_gradient():
+    w = inputs.custom(1, 2, 2, 256, 256, 128, True, True, seed=12)
+    t = inputs.make(w, device="cuda")
+    for mode in (1, 2):
+        kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q1"], t["k1"], causal=True)
+        dq, dk = binding.bwd(mode, t["q1"], t["k1"], t["q1"], t["k1"], kl, l1, l2, t["dkl"], causal=True)
+        torch.cuda.synchronize()
+        assert dq.abs().max().item() == 0 and dk.abs().max().item() == 0
+
+
+def test_extra_memory_is_only_the_workspace():
+    w = inputs.custom(1, 8, 8, 2048, 2048, 128, True, True, seed=9)
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], causal=True)
+    n = binding.streamkl_bwd_workspace_bytes(1, 8, 2048, 128) // 4
+    ws = torch.empty(n, device="cuda")
+    out = (torch.empty_like(t["q1"]), torch.empty_like(t["k1"]))
+    binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], causal=True, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], causal=True, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 >= free0
+
+
+def sampled_check(name, mode, causal=None, heads_for_dk=1, rows_per_head=32, keys_per_head=48):
+    base = inputs.WORKLOADS[name]
+    w = base if causal is None else inputs.variant(base, causal=causal)
+    t = inputs.make(w, device="cuda")
+    dq, dk = gpu_bwd(t, w, mode)
+    h = host(t)
+    rng = np.random.default_rng(7 + mode)
+    d = w.d
+    # dQ: sampled rows of every (b, head); each oracle row needs only its own row
+    rows = np.concatenate([bh * w.NQ + rng.choice(w.NQ, rows_per_head, replace=False)
+                           for bh in range(w.B * w.Hq)])
+    odq = oracle.bwd_dq_rows(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], rows,
+                             scale=w.scale, causal=w.causal)
+    gdq = dq.reshape(-1, d)[rows]
+    e = rel_l2(gdq.reshape(w.B * w.Hq, rows_per_head, d)[None], odq.reshape(w.B * w.Hq, rows_per_head, d)[None], axes=(2, 3))
+    assert e.max() <= GRAD_TOL, "%s dQ rel-L2 %.3g" % (name, e.max())
+    # dK: sampled keys of the first and last (b, KV head)
+    units = [0, w.B * w.Hkv - 1][:heads_for_dk] if heads_for_dk < 2 else [0, w.B * w.Hkv - 1]
+    keys = np.concatenate([u * w.NK + rng.choice(w.NK, keys_per_head, replace=False) for u in units])
+    odk = oracle.bwd_dk_keys(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], keys,
+                             scale=w.scale, causal=w.causal)
+    gdk = dk.reshape(-1, d)[keys]
+    e = rel_l2(gdk.reshape(len(units), keys_per_head, d)[None], odk.reshape(len(units), keys_per_head, d)[None], axes=(2, 3))
+    assert e.max() <= GRAD_TOL, "%s dK rel-L2 %.3g" % (name, e.max())
+    assert np.all(np.isfinite(dq)) and np.all(np.isfinite(dk))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_size_b2h8n4k_mode1(causal):
+    sampled_check("b2h8n4k", 1, causal=causal, heads_for_dk=2)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_full_size_headline(mode):
+    sampled_check("headline", mode, heads_for_dk=1)
+
+
+def test_full_size_gqa_mode2():
+    sampled_check("gqa", 2, heads_for_dk=1, rows_per_head=16, keys_per_head=32)
