@@ -226,6 +226,8 @@ def run_gpu(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     binding.load()
     base = inputs.WORKLOADS[WORKLOAD]
+    if args.heads != base.Hq:  # reduced-head case for profiler captures only
+        base = inputs.variant(base, Hq=args.heads, Hkv=args.heads)
     w = inputs.variant(base, seed=base.seed + 1000 * rank)  # own batch per rank
     t = inputs.make(w, device=dev)
     B, Hq, NQ, d = w.B, w.Hq, w.NQ, w.d
@@ -352,8 +354,9 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "B1 H32 NQ=NK=16384 d128 causal shared-K (headline); step = "
-                               "forward + backward P1-fixed + backward P2-fixed",
+        "config": {"workload": "B1 H%d NQ=NK=16384 d128 causal shared-K (%s); step = "
+                               "forward + backward P1-fixed + backward P2-fixed"
+                               % (Hq, "headline" if Hq == 32 else "reduced heads"),
                    "global_batch": world * B, "seq_len": NQ, "heads": Hq, "head_dim": d,
                    "parallelism": "dp%d (independent batch per GPU, no collective)" % world,
                    "l2": "inputs (3 x 128 MiB bf16) larger than the 126 MB L2; no flush"},
@@ -389,16 +392,18 @@ def run_gpu(args):
 
 
 def load_traffic(kernel):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or None."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
-        return None
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary
+    (profiles/dram_traffic.txt, lines "<call> <bytes>"), or None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         with open(p) as f:
-            d = json.load(f)
-        return d.get(kernel)
+            for line in f:
+                parts = line.split()
+                if len(parts) == 2 and not line.startswith("#") and parts[0] == kernel:
+                    return int(parts[1])
     except (OSError, ValueError):
         return None
+    return None
 
 
 def main():
@@ -409,6 +414,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU-oracle baseline leg")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    ap.add_argument("--heads", type=int, default=32,
+                    help="query/KV heads (32 = the headline workload; fewer only for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
