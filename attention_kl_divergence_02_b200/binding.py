@@ -26,6 +26,7 @@ EXPORTS = (
     "streamkl_fwd",
     "streamkl_bwd",
     "streamkl_bwd_workspace_bytes",
+    "streamkl_bwd_noalloc",
     "streamkl_status_string",
     "streamkl_device_status",
     "streamkl_last_cuda_error",
@@ -60,6 +61,9 @@ def load(path=None):
     lib.streamkl_bwd.argtypes = ([i, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
                                   vp, vp, vp, sz, vp])
     lib.streamkl_bwd.restype = i
+    lib.streamkl_bwd_noalloc.argtypes = ([i, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                          vp, vp, vp])
+    lib.streamkl_bwd_noalloc.restype = i
     lib.streamkl_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.streamkl_bwd_workspace_bytes.restype = sz
     lib.streamkl_status_string.argtypes = [i]
@@ -105,6 +109,22 @@ def streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, 
                                _ptr(lse1), _ptr(lse2), _ptr(dkl), B, Hq, Hkv, NQ, NK, d,
                                float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
                                _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+# Built-in scratch of streamkl_bwd_noalloc (STREAMKL_NOALLOC_SCRATCH_BYTES in the header).
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def streamkl_bwd_noalloc(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
+                         causal, dq, dk, stream=None):
+    """Backward without a workspace argument, for callers that may not allocate device
+    memory: the library's fixed 32 MiB built-in buffer holds the dQ accumulator.  Calls
+    that can overlap on the GPU share that buffer and race; larger problems return
+    ERR_UNSUPPORTED."""
+    return load().streamkl_bwd_noalloc(int(mode), _ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(kl),
+                                       _ptr(lse1), _ptr(lse2), _ptr(dkl), B, Hq, Hkv, NQ, NK, d,
+                                       float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
+                                       _stream(stream))
 
 
 def streamkl_bwd_workspace_bytes(B, Hq, NQ, d):

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "streamkl.h"
 #include "sm100.cuh"
@@ -232,3 +233,66 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation backward
+// The scratch buffer behind streamkl_bwd_noalloc: a fixed-size static device array, so the
+// entry point never allocates.  Host code must not pass `g_noalloc_dq_scratch` itself to a
+// kernel (on the host that name is only a stand-in for the symbol); it passes the device
+// address that cudaGetSymbolAddress returns, looked up once per device.
+static __device__ __align__(256) float g_noalloc_dq_scratch[STREAMKL_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (first call per device does
+// the lookup with that device current).  Returns nullptr and sets the error text on failure.
+float* noalloc_scratch() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "device %d beyond the %d supported",
+                 dev, kMaxDevices);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_dq_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int streamkl_bwd_noalloc(int mode, const uint16_t* q1, const uint16_t* k1,
+                                    const uint16_t* q2, const uint16_t* k2, const float* kl,
+                                    const float* lse1, const float* lse2, const float* dkl, int B,
+                                    int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                                    uint16_t* dq, uint16_t* dk, void* stream) {
+    if (mode != 1 && mode != 2) return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    const size_t need = streamkl_bwd_workspace_bytes(B, Hq, NQ, d);
+    if (need == 0 || need > STREAMKL_NOALLOC_SCRATCH_BYTES) {
+        snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
+                 "streamkl_bwd_noalloc: needs %zu bytes of scratch, the built-in buffer holds %zu",
+                 need, (size_t)STREAMKL_NOALLOC_SCRATCH_BYTES);
+        return STREAMKL_ERR_UNSUPPORTED;
+    }
+    float* ws = noalloc_scratch();
+    if (!ws) return STREAMKL_ERR_CUDA;
+    return streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
+                        causal, dq, dk, ws, need, stream);
+}

@@ -100,6 +100,38 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
                  int causal, uint16_t* dq, uint16_t* dk, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/*
+ * Size of the library's built-in backward scratch buffer (see streamkl_bwd_noalloc).
+ */
+#define STREAMKL_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * Backward that allocates nothing and takes no workspace argument.  This entry point has
+ * no counterpart in the StreamKL papers; it exists for callers that may not allocate
+ * device memory at all -- for example code running inside a framework whose allocator
+ * owns all of the GPU's memory and forbids side allocations, a service whose device-memory
+ * budget is fixed once it has started, or a latency-critical path that cannot afford the
+ * device-wide synchronisation that cudaMalloc/cudaFree can cause.
+ *
+ * Same arguments, semantics and outputs as streamkl_bwd, minus workspace/workspace_bytes:
+ * the fp32 dQ accumulator lives in a fixed STREAMKL_NOALLOC_SCRATCH_BYTES (32 MiB) buffer
+ * compiled into the library as a static device array.  Every GPU on which the library is
+ * loaded holds that buffer until the process exits.
+ *  - Sizes whose workspace (streamkl_bwd_workspace_bytes) exceeds the buffer return
+ *    STREAMKL_ERR_UNSUPPORTED and launch nothing; use streamkl_bwd for those.
+ *  - The first call on each device looks up the buffer's device address (a one-time
+ *    set-up done with that device current); make that first call before any stream
+ *    capture begins on the device.
+ *  - All calls on a device share the one buffer; it is cleared at the start of every call,
+ *    so leftover contents do not matter, but two calls that can run at the same time on
+ *    the GPU (different streams, no ordering between them) race on it and give undefined
+ *    results.  Order such calls on one stream or with events.
+ */
+int streamkl_bwd_noalloc(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
+                         const uint16_t* k2, const float* kl, const float* lse1, const float* lse2,
+                         const float* dkl, int B, int Hq, int Hkv, int NQ, int NK, int d,
+                         float scale, int causal, uint16_t* dq, uint16_t* dk, void* stream);
+
 /* Static text for a status code (never NULL). */
 const char* streamkl_status_string(int status);
 
