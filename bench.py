@@ -55,6 +55,29 @@ def host_cores():
         return os.cpu_count() or 1
 
 
+# ------------------------------------------------------------------ multi-rank host logic
+def rank_workload(base, rank):
+    """Weak scaling: every rank gets its own batch of the same workload (own seed)."""
+    from attention_kl_divergence_02_b200 import inputs
+    return inputs.variant(base, seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of timings over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    x = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return x.tolist()
+
+
+def job_tflops(world, flops_per_rank_step, ms_per_step):
+    """Whole-job throughput: every rank's work divided by the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -157,10 +180,16 @@ def cpu_baseline(w, target_s=15.0):
     oracle.build()
     cores = oracle.num_threads()
     _host_inputs(w)
-    probe_rows = max(8, 2 * cores)
-    dt, _ = oracle_sample(w, probe_rows, seed=1)
-    n = int(min(w.B * w.Hq * w.NQ, max(probe_rows, probe_rows * target_s / max(dt, 1e-3))))
-    dt, flops = oracle_sample(w, n, seed=2)
+    total_rows = w.B * w.Hq * w.NQ
+    n = max(8, 2 * cores)
+    dt, flops = oracle_sample(w, n, seed=1)
+    # grow the sample until it takes at least 2/3 of the target (small probes overstate the
+    # per-row cost: too few rows per thread)
+    for it in range(4):
+        if dt >= 0.66 * target_s or n >= total_rows:
+            break
+        n = int(min(total_rows, max(n + 1, n * target_s / max(dt, 1e-3))))
+        dt, flops = oracle_sample(w, n, seed=2 + it)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": "%d random query rows of the %s workload (all their valid keys): forward "
                       "+ both backward settings (dQ rows) in the fp64 C oracle, OpenMP over rows; "
@@ -228,7 +257,7 @@ def run_gpu(args):
     base = inputs.WORKLOADS[WORKLOAD]
     if args.heads != base.Hq:  # reduced-head case for profiler captures only
         base = inputs.variant(base, Hq=args.heads, Hkv=args.heads)
-    w = inputs.variant(base, seed=base.seed + 1000 * rank)  # own batch per rank
+    w = rank_workload(base, rank)
     t = inputs.make(w, device=dev)
     B, Hq, NQ, d = w.B, w.Hq, w.NQ, w.d
     stream = torch.cuda.current_stream()
@@ -284,13 +313,10 @@ def run_gpu(args):
     f_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     b1_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     b2_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
-    if world > 1:
-        x = torch.tensor([total_ms, f_ms, b1_ms, b2_ms], device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        total_ms, f_ms, b1_ms, b2_ms = x.tolist()
+    total_ms, f_ms, b1_ms, b2_ms = max_over_ranks([total_ms, f_ms, b1_ms, b2_ms], device=dev)
     ms_step = total_ms / args.steps
     step_flops = w.fwd_flops() + 2 * w.bwd_flops()
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, step_flops, ms_step)
 
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = None
@@ -334,12 +360,8 @@ def run_gpu(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / ne
-        if world > 1:
-            x = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(x, op=dist.ReduceOp.MAX)
-            e_ms = x.item()
-        e2e = {"value": world * step_flops / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e_ms = max_over_ranks([a.elapsed_time(b) / ne], device=dev)[0]
+        e2e = {"value": job_tflops(world, step_flops, e_ms), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     peaks, peak_src = load_peaks()
