@@ -17,8 +17,12 @@
 //                 shared tile that serves both MMAs below
 //   tensor core : dK += dS^T Q_free   (TMEM accumulator over all visits: no atomics)
 //                 dQp  = dS K_free    (TMEM, lane = query row)
-//   4 warpgroups: dQp added into the fp32 dQ workspace with vector atomics (the live rows
-//                 of the workspace stay resident in L2)
+//   4 warpgroups: dQp staged through shared memory and added into the fp32 dQ workspace
+//                 with bulk L2 reductions (cp.reduce.async.bulk .add.f32), off the L1 path
+// The workspace is private to the library and tile-blocked: one contiguous 128 x d block
+// per (batch, head, query tile), laid out in the order the warps hold it
+// ([warpgroup][lane quarter][4-column group][lane][4]), so that each warp's share is one
+// contiguous range; the convert kernel turns it into row-major bf16 dQ.
 // The MMA issuer looks one visit ahead: S of visit n+1 runs on the tensor core while the
 // warpgroups turn S of visit n into dS (needs two query stages in shared memory).
 //
@@ -60,8 +64,9 @@ struct BwdCfg {
     static constexpr int kK = 0;                                   // key tile i at kK + i*kTile
     static constexpr int kQ = kNK * kTile;                         // stage s: Q1 at kQ + s*2*kTile, Q2 after
     static constexpr int kDS = kQ + kQS * 2 * kTile;               // dS^T tile, 128 x 128 bf16
-    static constexpr int kCst = kDS + 128 * 128 * 2;               // per-query constants [16 warps][32] float4
-    static constexpr int kBar = kCst + 4 * kBwdWG * 32 * 16;
+    static constexpr int kStage = kDS + 128 * 128 * 2;             // dQ staging, 2 KiB per compute warp
+    static constexpr int kStageWarp = 2048;
+    static constexpr int kBar = kStage + 4 * kBwdWG * kStageWarp;
     static constexpr int K_FULL = 0;
     static constexpr int Q_FULL = 1;                // + s
     static constexpr int Q_EMPTY = 1 + kQS;         // + s
@@ -104,6 +109,24 @@ struct BwdSchedule {
         }
     }
 };
+
+// dst[0..bytes) += src[0..bytes) in L2 (fp32 add), read from shared memory by the bulk copy
+// engine; completion tracked by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 ::"l"(dst), "r"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// This thread's bulk groups have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's bulk groups have completed (global writes done).
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
@@ -325,23 +348,42 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         const float sl2 = p.sl2;
         const float scale = p.scale;
         const float LOG2E = 1.4426950408889634f;
-        float4* cst = reinterpret_cast<float4*>(smem + C::kCst);
         uint8_t* ds_tile = smem + C::kDS;
         // this thread's 64 bytes of the dS^T row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
         uint8_t* ds_row = ds_tile + (wg >> 1) * C::kBox + r * 128;
+        // this warp's dQ staging slot: [4-column group (4)][lane (32)][4 floats] = 2 KiB
+        float4* stage = reinterpret_cast<float4*>(smem + C::kStage + (warp - 4) * C::kStageWarp);
+        const uint32_t stage_s = smem_u32(stage);
+        constexpr int kCols = D / 4;          // dQ / dK columns per warpgroup
+        constexpr int kRounds = D / 64;       // 2 KiB staging rounds per visit
         bool ok = true;
-        int prev_bh = 0, prev_q0 = 0;
-        auto drain_dq = [&](int n_done, int bh_, int q0_) -> bool {
+        int prev_bh = 0, prev_qt = 0;
+        // Move this warp's share of the dQ partial of an earlier visit into the workspace
+        // block of (bh_, qt_): TMEM -> registers -> staging slot -> bulk L2 reduction.
+        auto flush_dq = [&](int n_done, int bh_, int qt_) -> bool {
             if (!mbar_wait(BAR(C::DQ_FULL), n_done & 1, abort_flag)) return false;
             tc_fence_after();
-            float v[D / 4];
-            tmem_ld_quarter<D>(lane_base + C::kColDQ + wg * (D / 4), v);
-            const int q = q0_ + r;
-            if (q < p.NQ) {
-                float4* dst = reinterpret_cast<float4*>(p.dq_ws + ((size_t)bh_ * p.NQ + q) * D + wg * (D / 4));
+            float v[kCols];
+            tmem_ld_quarter<D>(lane_base + C::kColDQ + wg * kCols, v);
+            tc_fence_before();
+            mbar_arrive(BAR(C::DQ_FREE));
+            float* blk = p.dq_ws + ((size_t)bh_ * p.nqt + qt_) * (128 * D) +
+                         (size_t)(wg * 4 + quarter) * (32 * kCols);
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    atomicAdd(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+            for (int rd = 0; rd < kRounds; ++rd) {
+                if (lane == 0) bulk_wait_read_all();   // the slot's previous contents were read
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int c = (rd * 4 + g) * 4;
+                    stage[g * 32 + lane] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_reduce_add_f32(blk + rd * 512, stage_s, C::kStageWarp);
+                    bulk_commit();
+                }
             }
             return true;
         };
@@ -350,23 +392,18 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             sched.visit(n, h, qt);
             const int bh = b * p.Hq + h;
             const int q0 = qt * 128;
-            // per-query constants of this warpgroup's 32 columns, one copy per warp (only
-            // warp-level syncs: no barrier that an aborting sibling warp could leave hanging)
-            float4* cbuf = cst + (warp - 4) * 32;
+            // per-query constants of query q0 + 32*wg + lane, broadcast with shuffles below:
+            // ca = LSE1*log2(e), cb = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2), cg = g
+            float ca = 0.f, cb = 0.f, cg = 0.f;
             {
                 const int q = q0 + wg * 32 + lane;
-                float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (q < p.NQ) {
                     const size_t o = (size_t)bh * p.NQ + q;
                     const float L1 = p.lse1[o], L2 = p.lse2[o];
-                    c.x = L1 * LOG2E;
-                    c.y = L2 * LOG2E;
-                    c.z = p.dkl[o];
-                    c.w = mode1 ? 0.f : (L2 - L1 - p.kl[o]);
+                    ca = L1 * LOG2E;
+                    cb = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
+                    cg = p.dkl[o];
                 }
-                __syncwarp();          // the previous visit's reads of cbuf are done
-                cbuf[lane] = c;
-                __syncwarp();
             }
             if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
                 ok = false;
@@ -389,16 +426,18 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 float ds[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float4 c = cbuf[k + e];
+                    const float a = __shfl_sync(0xffffffffu, ca, k + e);
+                    const float bw = __shfl_sync(0xffffffffu, cb, k + e);
+                    const float gq = __shfl_sync(0xffffffffu, cg, k + e);
                     const float x = __uint_as_float(xa[k + e]);
                     const float y = __uint_as_float(ya[k + e]);
-                    const float p1 = ex2(fmaf(x, sl2, -c.x));
+                    const float p1 = ex2(fmaf(x, sl2, -a));
                     float v;
                     if (mode1) {
-                        const float p2 = ex2(fmaf(y, sl2, -c.y));
-                        v = c.z * (p2 - p1);
+                        const float p2 = ex2(fmaf(y, sl2, -bw));
+                        v = gq * (p2 - p1);
                     } else {
-                        v = c.z * p1 * fmaf(scale, x - y, c.w);
+                        v = gq * p1 * fmaf(scale, x - y, bw);
                     }
                     if ((diag && r > qoff + k + e) || !key_ok) v = 0.f;
                     ds[e] = v;
@@ -418,24 +457,20 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             }
             fence_async_smem();
             mbar_arrive(BAR(C::DS_FULL));
-            if (n > 0) {
-                if (!drain_dq(n - 1, prev_bh, prev_q0)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_before();
-                mbar_arrive(BAR(C::DQ_FREE));
+            if (n > 0 && !flush_dq(n - 1, prev_bh, prev_qt)) {
+                ok = false;
+                break;
             }
             prev_bh = bh;
-            prev_q0 = q0;
+            prev_qt = qt;
         }
-        if (ok && N > 0) ok = drain_dq(N - 1, prev_bh, prev_q0);
+        if (ok && N > 0) ok = flush_dq(N - 1, prev_bh, prev_qt);
         if (ok && mbar_wait(BAR(C::DK_FULL), 0, abort_flag)) {
             tc_fence_after();
-            float v[D / 4];
-            tmem_ld_quarter<D>(lane_base + C::kColDK + wg * (D / 4), v);
+            float v[kCols];
+            tmem_ld_quarter<D>(lane_base + C::kColDK + wg * kCols, v);
             if (k0 + r < p.NK) {
-                uint4* dst = reinterpret_cast<uint4*>(p.dk + ((size_t)bhk * p.NK + k0 + r) * D + wg * (D / 4));
+                uint4* dst = reinterpret_cast<uint4*>(p.dk + ((size_t)bhk * p.NK + k0 + r) * D + wg * kCols);
 #pragma unroll
                 for (int k = 0; k < D / 32; ++k)
                     dst[k] = make_uint4(pack_bf16(v[8 * k] * scale, v[8 * k + 1] * scale),
@@ -444,6 +479,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                                         pack_bf16(v[8 * k + 6] * scale, v[8 * k + 7] * scale));
             }
         }
+        // every bulk reduction this warp started has landed before the CTA exits
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -455,15 +493,35 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #undef BAR
 }
 
-// dq[i] = bf16(ws[i] * scale), eight elements per thread per step.
+// dq = bf16(scale * ws), un-blocking the tile-blocked workspace.  One thread = one query
+// row's D/4 columns of one warpgroup slice: it reads D/16 float4 (coalesced across the 32
+// lanes of the block) and writes D/2 contiguous bytes of its dQ row.
+template <int D>
 __global__ void __launch_bounds__(256)
-streamkl_dq_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dq, size_t n8, float scale) {
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
-        const float4 a = reinterpret_cast<const float4*>(ws)[2 * i];
-        const float4 c = reinterpret_cast<const float4*>(ws)[2 * i + 1];
-        reinterpret_cast<uint4*>(dq)[i] =
-            make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
-                       pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+streamkl_dq_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dq, int BH, int NQ,
+                           int nqt, float scale) {
+    constexpr int kCols = D / 4;
+    const size_t total = (size_t)BH * nqt * 512;   // (bh, tile, wg, quarter, lane)
+    for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
+         t += (size_t)gridDim.x * blockDim.x) {
+        const int lane = (int)(t & 31);
+        const int quarter = (int)((t >> 5) & 3);
+        const int wg = (int)((t >> 7) & 3);
+        const size_t blk = t >> 9;                 // bh * nqt + qt
+        const int qt = (int)(blk % nqt);
+        const size_t bh = blk / nqt;
+        const int q = qt * 128 + quarter * 32 + lane;
+        if (q >= NQ) continue;
+        const float4* src = reinterpret_cast<const float4*>(
+            ws + blk * (128 * D) + (size_t)(wg * 4 + quarter) * (32 * kCols)) + lane;
+        uint4* dst = reinterpret_cast<uint4*>(dq + (bh * NQ + q) * D + wg * kCols);
+#pragma unroll
+        for (int k = 0; k < kCols / 8; ++k) {
+            const float4 a = src[(2 * k) * 32];
+            const float4 c = src[(2 * k + 1) * 32];
+            dst[k] = make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
+                                pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+        }
     }
 }
 

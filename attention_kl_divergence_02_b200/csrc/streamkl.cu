@@ -110,10 +110,11 @@ int launch_bwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
     kern<<<grid, skl::kBwdThreads, smem, st>>>(q1, q2, k1, k2, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_bwd launch");
-    const size_t n8 = ws_bytes / sizeof(float) / 8;
-    size_t blocks = (n8 + 255) / 256;
+    const size_t threads = (size_t)p.B * p.Hq * p.nqt * 512;
+    size_t blocks = (threads + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    skl::streamkl_dq_convert_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.dq_ws, dq, n8, p.scale);
+    skl::streamkl_dq_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(p.dq_ws, dq, p.B * p.Hq,
+                                                                        p.NQ, p.nqt, p.scale);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dq convert launch");
     return STREAMKL_OK;
@@ -186,7 +187,8 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
 
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d) {
     if (B < 1 || Hq < 1 || NQ < 1 || (d != 64 && d != 128)) return 0;
-    return (size_t)B * Hq * NQ * d * sizeof(float);
+    const size_t rows = (size_t)(NQ + 127) / 128 * 128;   // whole 128-row query tiles
+    return (size_t)B * Hq * rows * d * sizeof(float);
 }
 
 int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,

@@ -68,8 +68,8 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
                  float* kl, float* lse1, float* lse2, void* stream);
 
 /*
- * Bytes of fp32 workspace streamkl_bwd needs: B*Hq*NQ*d*4 (the dQ accumulator).  Returns
- * 0 for sizes outside the supported range.
+ * Bytes of fp32 workspace streamkl_bwd needs: B*Hq*ceil(NQ/128)*128*d*4 (the dQ
+ * accumulator, whole 128-row query tiles).  Returns 0 for sizes outside the supported range.
  */
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d);
 

@@ -45,7 +45,8 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_bytes(lib):
     assert binding.streamkl_bwd_workspace_bytes(1, 32, 16384, 128) == 32 * 16384 * 128 * 4
-    assert binding.streamkl_bwd_workspace_bytes(2, 3, 5, 64) == 2 * 3 * 5 * 64 * 4
+    assert binding.streamkl_bwd_workspace_bytes(2, 3, 5, 64) == 2 * 3 * 128 * 64 * 4   # whole tiles
+    assert binding.streamkl_bwd_workspace_bytes(1, 1, 129, 128) == 256 * 128 * 4
     assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 96) == 0
     assert binding.streamkl_bwd_workspace_bytes(0, 1, 1, 64) == 0
 
@@ -83,7 +84,7 @@ def test_fwd_rejects_on_host(lib, kw, want):
 def bwd_call(**kw):
     args = dict(mode=1, q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, kl=FAKE, lse1=FAKE, lse2=FAKE,
                 dkl=FAKE, B=1, Hq=2, Hkv=1, NQ=8, NK=8, d=64, scale=0.125, causal=0, dq=FAKE,
-                dk=FAKE, workspace=FAKE, workspace_bytes=2 * 8 * 64 * 4, stream=0)
+                dk=FAKE, workspace=FAKE, workspace_bytes=2 * 128 * 64 * 4, stream=0)
     args.update(kw)
     return binding.streamkl_bwd(**args)
 
@@ -93,7 +94,7 @@ def bwd_call(**kw):
     (dict(mode=3), binding.ERR_INVALID_ARG),
     (dict(dq=None), binding.ERR_INVALID_ARG),
     (dict(workspace=None), binding.ERR_INVALID_ARG),
-    (dict(workspace_bytes=2 * 8 * 64 * 4 - 4), binding.ERR_INVALID_ARG),
+    (dict(workspace_bytes=2 * 128 * 64 * 4 - 4), binding.ERR_INVALID_ARG),
     (dict(d=32), binding.ERR_UNSUPPORTED),
     (dict(causal=1, NK=7), binding.ERR_UNSUPPORTED),
     (dict(dk=FAKE + 2), binding.ERR_UNSUPPORTED),
