@@ -12,11 +12,13 @@
 // tile of every query head in the KV group that can see it (causal: from the diagonal
 // on), so each (query tile, key tile) pair is visited exactly once ("Fusão de Kernel").
 // Per visit n:
-//   tensor core : S1^T = K1 Q1^T, S2^T = K2 Q2^T           (TMEM, lane = key)
-//   4 warpgroups: dS^T for 32 query columns each -> bf16, written once into a swizzled
-//                 shared tile that serves both MMAs below
-//   tensor core : dK += dS^T Q_free   (TMEM accumulator over all visits: no atomics)
-//                 dQp  = dS K_free    (TMEM, lane = query row)
+//   tensor core : S1 = Q1 K1^T, S2 = Q2 K2^T               (TMEM, lane = query row)
+//   4 warpgroups: dS for 32 key columns each (thread = query row, so the row's LSEs, KL
+//                 and g sit in registers) -> bf16, written once into a swizzled shared
+//                 tile [query][key] that serves both MMAs below
+//   tensor core : dK += dS^T Q_free   (dS read MN-major; TMEM accumulator over all
+//                                      visits, lane = key: no atomics)
+//                 dQp  = dS K_free    (dS read K-major; TMEM, lane = query row)
 //   4 warpgroups: dQp staged through shared memory and added into the fp32 dQ workspace
 //                 with bulk L2 reductions (cp.reduce.async.bulk .add.f32), off the L1 path
 // The workspace is private to the library and tile-blocked: one contiguous 128 x d block
@@ -163,7 +165,36 @@ __device__ __forceinline__ void tmem_ld_quarter(uint32_t taddr, float (&v)[D / 4
     }
 }
 
-template <int D, bool SHARED_K>
+// dS of one query row over 32 key columns, packed to bf16 pairs.  x = S1 raw, y = S2 raw;
+// a = LSE1*log2(e); b = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2); g = upstream
+// gradient.  With MASKED, columns k >= lim are zero.
+template <int MODE, bool MASKED>
+__device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
+                                         float sl2, float scale, float a, float b, float g,
+                                         int lim, uint32_t (&packed)[16]) {
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float x = __uint_as_float(xa[k + e]);
+            const float y = __uint_as_float(ya[k + e]);
+            const float p1 = ex2(fmaf(x, sl2, -a));
+            float v;
+            if (MODE == 1) {
+                const float p2 = ex2(fmaf(y, sl2, -b));
+                v = g * (p2 - p1);
+            } else {
+                v = g * p1 * fmaf(scale, x - y, b);
+            }
+            if (MASKED && k + e >= lim) v = 0.f;
+            ds[e] = v;
+        }
+        packed[k >> 1] = pack_bf16(ds[0], ds[1]);
+    }
+}
+
+template <int D, bool SHARED_K, int MODE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
@@ -189,7 +220,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int k0 = kt * 128;
     const BwdSchedule sched(p, hk, kt);
     const int N = sched.count;
-    const bool mode1 = (p.mode == 1);
+    constexpr bool mode1 = (MODE == 1);
     // the free distribution's operands: mode 1 -> (Q2, K2), mode 2 -> (Q1, K1)
     const uint32_t kfree = sb + C::kK + ((SHARED_K || !mode1) ? 0 : C::kTile);
     const uint32_t k2tile = sb + C::kK + (SHARED_K ? 0 : C::kTile);
@@ -262,9 +293,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // K-major A and B
-            constexpr uint32_t idK = idesc_bf16(128, D, 0, 1);     // dS^T K-major, Q MN-major
-            constexpr uint32_t idQ = idesc_bf16(128, D, 1, 1);     // dS MN-major, K MN-major
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // Q, K both K-major
+            constexpr uint32_t idK = idesc_bf16(128, D, 1, 1);     // dS^T MN-major, Q MN-major
+            constexpr uint32_t idQ = idesc_bf16(128, D, 0, 1);     // dS K-major, K MN-major
             auto issue_S = [&](int n) {
                 const int s = n % C::kQS;
                 const uint32_t q1s = sb + C::kQ + s * 2 * C::kTile;
@@ -272,14 +303,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(sb + C::kK + off, 16, 1024),
-                                sw128_desc(q1s + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(q1s + off, 16, 1024),
+                                sw128_desc(sb + C::kK + off, 16, 1024), idS, k > 0);
                 }
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(k2tile + off, 16, 1024),
-                                sw128_desc(q2s + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(q2s + off, 16, 1024),
+                                sw128_desc(k2tile + off, 16, 1024), idS, k > 0);
                 }
                 mma_commit(BAR(C::S_FULL));
             };
@@ -288,15 +319,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 const uint32_t qf = sb + C::kQ + s * 2 * C::kTile + (mode1 ? C::kTile : 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDK,
-                                sw128_desc(sb + C::kDS + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
+                    mma_bf16_ss(tmem + C::kColDK, sw128_desc(sb + C::kDS + k * 2048, C::kBox, 1024),
                                 sw128_desc(qf + k * 2048, C::kBox, 1024), idK, (n > 0 || k > 0));
                 }
             };
             auto issue_dQ = [&]() {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDQ, sw128_desc(sb + C::kDS + k * 2048, C::kBox, 1024),
+                    mma_bf16_ss(tmem + C::kColDQ,
+                                sw128_desc(sb + C::kDS + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
                                 sw128_desc(kfree + k * 2048, C::kBox, 1024), idQ, k > 0);
                 }
             };
@@ -341,9 +372,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         }
     } else if (warp >= 4) {
         // ================================================================ compute warpgroups
-        const int wg = (warp - 4) >> 2;         // query columns [32*wg, 32*wg + 32)
+        const int wg = (warp - 4) >> 2;         // key columns [32*wg, 32*wg + 32)
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;      // TMEM lane: key row (S, dK) or query row (dQ)
+        const int r = quarter * 32 + lane;      // TMEM lane: query row (S, dQ) or key row (dK)
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.sl2;
         const float scale = p.scale;
@@ -392,11 +423,11 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             sched.visit(n, h, qt);
             const int bh = b * p.Hq + h;
             const int q0 = qt * 128;
-            // per-query constants of query q0 + 32*wg + lane, broadcast with shuffles below:
-            // ca = LSE1*log2(e), cb = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2), cg = g
+            // this thread's query row: ca = LSE1*log2(e), cb = LSE2*log2(e) (mode 1) or
+            // LSE2 - LSE1 - KL (mode 2), cg = g; rows past NQ get g = 0 (their dS is 0)
             float ca = 0.f, cb = 0.f, cg = 0.f;
             {
-                const int q = q0 + wg * 32 + lane;
+                const int q = q0 + r;
                 if (q < p.NQ) {
                     const size_t o = (size_t)bh * p.NQ + q;
                     const float L1 = p.lse1[o], L2 = p.lse2[o];
@@ -416,34 +447,20 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(BAR(C::S_FREE));
-            // dS^T[r, q] for the 32 query columns
-            const bool diag = p.causal && (qt == kt);
-            const bool key_ok = (k0 + r < p.NK);   // zero-filled key rows past NK get dS = 0
-            const int qoff = wg * 32;      // column offset within the query tile
-            uint32_t packed[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-                float ds[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float a = __shfl_sync(0xffffffffu, ca, k + e);
-                    const float bw = __shfl_sync(0xffffffffu, cb, k + e);
-                    const float gq = __shfl_sync(0xffffffffu, cg, k + e);
-                    const float x = __uint_as_float(xa[k + e]);
-                    const float y = __uint_as_float(ya[k + e]);
-                    const float p1 = ex2(fmaf(x, sl2, -a));
-                    float v;
-                    if (mode1) {
-                        const float p2 = ex2(fmaf(y, sl2, -bw));
-                        v = gq * (p2 - p1);
-                    } else {
-                        v = gq * p1 * fmaf(scale, x - y, bw);
-                    }
-                    if ((diag && r > qoff + k + e) || !key_ok) v = 0.f;
-                    ds[e] = v;
-                }
-                packed[k >> 1] = pack_bf16(ds[0], ds[1]);
+            // dS[r, key] for the 32 key columns.  Masked: keys past the diagonal of a causal
+            // diagonal tile and zero-filled keys past NK.
+            const int kc0 = wg * 32;               // first key column of this warpgroup
+            const bool need_mask = (p.causal && qt == kt) || (k0 + 128 > p.NK);
+            int lim = 32;                          // columns k < lim are valid keys
+            if (need_mask) {
+                lim = min(lim, p.NK - k0 - kc0);
+                if (p.causal && qt == kt) lim = min(lim, r - kc0 + 1);
             }
+            uint32_t packed[16];
+            if (need_mask)
+                ds_chunk<MODE, true>(xa, ya, sl2, scale, ca, cb, cg, lim, packed);
+            else
+                ds_chunk<MODE, false>(xa, ya, sl2, scale, ca, cb, cg, 32, packed);
             if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
                 ok = false;
                 break;

@@ -60,6 +60,17 @@ struct FwdCfg {
 };
 
 
+// Columns (bit k of a 32-column chunk) whose exponentials go to the FMA-pipe polynomial
+// instead of the exponential unit, for S1 and for S2: the two pipes then share the load.
+#ifndef SKL_FWD_EMU1
+#define SKL_FWD_EMU1 0u
+#endif
+#ifndef SKL_FWD_EMU2
+#define SKL_FWD_EMU2 0u
+#endif
+constexpr uint32_t kEmu1 = SKL_FWD_EMU1;
+constexpr uint32_t kEmu2 = SKL_FWD_EMU2;
+
 // Fold 32 columns of one row into the running scalars.  x = S1 raw scores, y = S2 raw.
 // `valid` has bit k set when column k is a valid key for this row.
 template <bool MASKED>
@@ -91,8 +102,10 @@ __device__ __forceinline__ void fold_chunk(const uint32_t (&xa)[32], const uint3
     float sl1[2] = {0.f, 0.f}, sl2v[2] = {0.f, 0.f}, sac[2] = {0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-        const float e1 = ex2(fmaf(x[k], sl2, -m1n));
-        const float e2 = ex2(fmaf(y[k], sl2, -m2n));
+        const float u1 = fmaf(x[k], sl2, -m1n);
+        const float u2 = fmaf(y[k], sl2, -m2n);
+        const float e1 = ((kEmu1 >> k) & 1u) ? ex2_poly(u1) : ex2(u1);
+        const float e2 = ((kEmu2 >> k) & 1u) ? ex2_poly(u2) : ex2(u2);
         float diff = x[k] - y[k];
         if (MASKED && !((valid >> k) & 1u)) diff = 0.f;
         sl1[k & 1] += e1;

@@ -101,7 +101,7 @@ template <int D, bool SHARED>
 int launch_bwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                const CUtensorMap& k2, const skl::BwdParams& p, int grid, size_t ws_bytes,
                uint16_t* dq, cudaStream_t st) {
-    auto kern = skl::streamkl_bwd_kernel<D, SHARED>;
+    auto kern = p.mode == 1 ? skl::streamkl_bwd_kernel<D, SHARED, 1> : skl::streamkl_bwd_kernel<D, SHARED, 2>;
     constexpr int smem = skl::BwdCfg<D, SHARED>::kSmem;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
