@@ -167,30 +167,42 @@ __device__ __forceinline__ void tmem_ld_quarter(uint32_t taddr, float (&v)[D / 4
 
 // dS of one query row over 32 key columns, packed to bf16 pairs.  x = S1 raw, y = S2 raw;
 // a = LSE1*log2(e); b = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2); g = upstream
-// gradient.  With MASKED, columns k >= lim are zero.
-template <int MODE, bool MASKED>
+// gradient.  FOLDED: g >= 0 has been folded into the exponents (a and, in mode 1, b
+// lowered by log2 g, so 2^(u - a) is already g*P) and g is not multiplied again.  Adjacent
+// columns are processed as fp32x2 pairs.  With MASKED, columns k >= lim are zero.
+template <int MODE, bool MASKED, bool FOLDED>
 __device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
                                          float sl2, float scale, float a, float b, float g,
                                          int lim, uint32_t (&packed)[16]) {
+    const float2 sl = make_float2(sl2, sl2);
+    const float2 na = make_float2(-a, -a);
+    const float2 nb = make_float2(-b, -b);
+    const float2 bb = make_float2(b, b);
+    const float2 gg = make_float2(g, g);
+    const float2 sc = make_float2(scale, scale);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int k = 0; k < 32; k += 2) {
-        float ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float x = __uint_as_float(xa[k + e]);
-            const float y = __uint_as_float(ya[k + e]);
-            const float p1 = ex2(fmaf(x, sl2, -a));
-            float v;
-            if (MODE == 1) {
-                const float p2 = ex2(fmaf(y, sl2, -b));
-                v = g * (p2 - p1);
-            } else {
-                v = g * p1 * fmaf(scale, x - y, b);
-            }
-            if (MASKED && k + e >= lim) v = 0.f;
-            ds[e] = v;
+    for (int pr = 0; pr < 16; ++pr) {
+        const float2 xk = make_float2(__uint_as_float(xa[2 * pr]), __uint_as_float(xa[2 * pr + 1]));
+        const float2 yk = make_float2(__uint_as_float(ya[2 * pr]), __uint_as_float(ya[2 * pr + 1]));
+        const float2 u1 = __ffma2_rn(xk, sl, na);
+        const float2 p1 = make_float2(ex2(u1.x), ex2(u1.y));
+        float2 v;
+        if (MODE == 1) {
+            const float2 u2 = __ffma2_rn(yk, sl, nb);
+            const float2 p2 = make_float2(ex2(u2.x), ex2(u2.y));
+            v = __ffma2_rn(p1, neg1, p2);                  // (g)P2 - (g)P1
+            if (!FOLDED) v = __fmul2_rn(v, gg);
+        } else {
+            const float2 r = __ffma2_rn(__ffma2_rn(yk, neg1, xk), sc, bb);   // scale(x-y) + b
+            v = __fmul2_rn(p1, r);
+            if (!FOLDED) v = __fmul2_rn(v, gg);
         }
-        packed[k >> 1] = pack_bf16(ds[0], ds[1]);
+        if (MASKED) {
+            if (2 * pr >= lim) v.x = 0.f;
+            if (2 * pr + 1 >= lim) v.y = 0.f;
+        }
+        packed[pr] = pack_bf16(v.x, v.y);
     }
 }
 
@@ -418,24 +430,34 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             }
             return true;
         };
+        // per-row statistics of visit n for this thread's query row
+        auto load_row_consts = [&](int n, float& ra, float& rb, float& rg) {
+            int h, qt;
+            sched.visit(n, h, qt);
+            const int q = qt * 128 + r;
+            ra = 0.f;
+            rb = 0.f;
+            rg = 0.f;
+            if (q < p.NQ) {
+                const size_t o = (size_t)(b * p.Hq + h) * p.NQ + q;
+                const float L1 = p.lse1[o], L2 = p.lse2[o];
+                ra = L1 * LOG2E;
+                rb = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
+                rg = p.dkl[o];
+            }
+        };
+        float na = 0.f, nb = 0.f, ng = 0.f;
+        if (N > 0) load_row_consts(0, na, nb, ng);
         for (int n = 0; n < N; ++n) {
             int h, qt;
             sched.visit(n, h, qt);
             const int bh = b * p.Hq + h;
             const int q0 = qt * 128;
             // this thread's query row: ca = LSE1*log2(e), cb = LSE2*log2(e) (mode 1) or
-            // LSE2 - LSE1 - KL (mode 2), cg = g; rows past NQ get g = 0 (their dS is 0)
-            float ca = 0.f, cb = 0.f, cg = 0.f;
-            {
-                const int q = q0 + r;
-                if (q < p.NQ) {
-                    const size_t o = (size_t)bh * p.NQ + q;
-                    const float L1 = p.lse1[o], L2 = p.lse2[o];
-                    ca = L1 * LOG2E;
-                    cb = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
-                    cg = p.dkl[o];
-                }
-            }
+            // LSE2 - LSE1 - KL (mode 2), cg = g; rows past NQ get g = 0 (their dS is 0).
+            // The next visit's values are loaded now and used one iteration later.
+            const float ca = na, cb = nb, cg = ng;
+            if (n + 1 < N) load_row_consts(n + 1, na, nb, ng);
             if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
                 ok = false;
                 break;
@@ -457,10 +479,22 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 if (p.causal && qt == kt) lim = min(lim, r - kc0 + 1);
             }
             uint32_t packed[16];
-            if (need_mask)
-                ds_chunk<MODE, true>(xa, ya, sl2, scale, ca, cb, cg, lim, packed);
-            else
-                ds_chunk<MODE, false>(xa, ya, sl2, scale, ca, cb, cg, 32, packed);
+            // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf
+            // makes a row with g = 0 give exactly 0)
+            if (!__any_sync(0xffffffffu, cg < 0.f)) {
+                const float lg = log2f(cg);
+                const float fa = ca - lg;
+                const float fb = mode1 ? cb - lg : cb;
+                if (need_mask)
+                    ds_chunk<MODE, true, true>(xa, ya, sl2, scale, fa, fb, cg, lim, packed);
+                else
+                    ds_chunk<MODE, false, true>(xa, ya, sl2, scale, fa, fb, cg, 32, packed);
+            } else {
+                if (need_mask)
+                    ds_chunk<MODE, true, false>(xa, ya, sl2, scale, ca, cb, cg, lim, packed);
+                else
+                    ds_chunk<MODE, false, false>(xa, ya, sl2, scale, ca, cb, cg, 32, packed);
+            }
             if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
                 ok = false;
                 break;

@@ -223,4 +223,27 @@ __device__ __forceinline__ float ex2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// ex2_poly on two values at once with packed fp32x2 arithmetic (one instruction per pair).
+__device__ __forceinline__ float2 ex2_poly2(float2 u) {
+    u.x = fmaxf(u.x, -126.0f);
+    u.y = fmaxf(u.y, -126.0f);
+    const float2 t = __fadd2_rn(u, make_float2(12582912.0f, 12582912.0f));
+    const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), u);
+    float2 p = __ffma2_rn(make_float2(9.570102207e-03f, 9.570102207e-03f), f,
+                          make_float2(5.591785908e-02f, 5.591785908e-02f));
+    p = __ffma2_rn(p, f, make_float2(2.402474433e-01f, 2.402474433e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.931217909e-01f, 6.931217909e-01f));
+    p = __ffma2_rn(p, f, make_float2(9.999992847e-01f, 9.999992847e-01f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// max of three floats in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 }  // namespace skl

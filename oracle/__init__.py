@@ -21,6 +21,7 @@ from .oracle import (  # noqa: F401
     bwd,
     bwd_dq_rows,
     bwd_dk_keys,
+    bwd_dk_keys_stats,
     num_threads,
     set_num_threads,
 )

@@ -45,8 +45,11 @@ def _load():
             lib.oracle_bwd.argtypes = [_i, _D, _D, _D, _D, _D] + shape + [_D, _D]
             lib.oracle_bwd_dq_rows.argtypes = [_i, _D, _D, _D, _D, _D] + shape + [_I64, ctypes.c_int64, _D]
             lib.oracle_bwd_dk_keys.argtypes = [_i, _D, _D, _D, _D, _D] + shape + [_I64, ctypes.c_int64, _D]
+            lib.oracle_bwd_dk_keys_stats.argtypes = ([_i, _D, _D, _D, _D, _D, _D, _D, _D] + shape +
+                                                     [_I64, ctypes.c_int64, _D])
             for f in ("oracle_fwd", "oracle_fwd_rows", "oracle_fwd_streaming", "oracle_bwd",
-                      "oracle_bwd_dq_rows", "oracle_bwd_dk_keys", "oracle_num_threads"):
+                      "oracle_bwd_dq_rows", "oracle_bwd_dk_keys", "oracle_bwd_dk_keys_stats",
+                      "oracle_num_threads"):
                 getattr(lib, f).restype = _i
             lib.oracle_set_num_threads.argtypes = [_i]
             lib.oracle_set_num_threads.restype = None
@@ -167,4 +170,24 @@ def bwd_dk_keys(mode, q1, k1, q2, k2, dkl, keys, scale=None, causal=False):
                                 _default_scale(d, scale), int(bool(causal)),
                                 keys.ctypes.data_as(_I64), keys.shape[0], out.ctypes.data_as(_D))
     _check(rc, "oracle_bwd_dk_keys")
+    return out
+
+
+def bwd_dk_keys_stats(mode, q1, k1, q2, k2, dkl, kl, lse1, lse2, keys, scale=None, causal=False):
+    """dK for flat key indices with every row's (KL, LSE1, LSE2) given as inputs
+    ([B,Hq,NQ] each) rather than recomputed: for sizes where the full statistics are out of
+    reach.  Only as independent as the statistics passed in."""
+    lib = _load()
+    B, Hq, Hkv, NQ, NK, d = _shape(q1, k1, q2, k2)
+    arrs = [_f64(x) for x in (q1, k1, q2, k2)]
+    st = [_f64(x) for x in (dkl, kl, lse1, lse2)]
+    for a, _ in st:
+        if a.shape != (B, Hq, NQ):
+            raise ValueError("row statistics must be [B,Hq,NQ]")
+    keys = np.ascontiguousarray(keys, dtype=np.int64)
+    out = np.empty((keys.shape[0], d))
+    rc = lib.oracle_bwd_dk_keys_stats(int(mode), *[p for _, p in arrs], *[p for _, p in st], B, Hq,
+                                      Hkv, NQ, NK, d, _default_scale(d, scale), int(bool(causal)),
+                                      keys.ctypes.data_as(_I64), keys.shape[0], out.ctypes.data_as(_D))
+    _check(rc, "oracle_bwd_dk_keys_stats")
     return out

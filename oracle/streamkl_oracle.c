@@ -459,6 +459,57 @@ int oracle_bwd_dk_keys(int mode, const double* q1, const double* k1, const doubl
     return rc;
 }
 
+/*
+ * dK for flat key indices like oracle_bwd_dk_keys, but with the row statistics (KL, LSE1,
+ * LSE2 of every row, [B*Hq*NQ]) taken as inputs instead of recomputed.  For sizes where
+ * recomputing every row's statistics is out of reach; the caller states where the
+ * statistics came from.
+ */
+int oracle_bwd_dk_keys_stats(int mode, const double* q1, const double* k1, const double* q2,
+                             const double* k2, const double* dkl, const double* KL,
+                             const double* L1, const double* L2, int B, int Hq, int Hkv, int NQ,
+                             int NK, int d, double scale, int causal, const int64_t* keys,
+                             int64_t nkeys, double* dk_keys) {
+    shape_t s = {B, Hq, Hkv, NQ, NK, d, causal, scale};
+    if (!shape_ok(&s) || (mode != 1 && mode != 2) || nkeys < 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t totalk = (int64_t)B * Hkv * NK;
+    for (int64_t t = 0; t < nkeys; ++t) if (keys[t] < 0 || keys[t] >= totalk) return -1;
+    const double* Qf = (mode == 1) ? q2 : q1;
+    memset(dk_keys, 0, sizeof(double) * (size_t)nkeys * d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nkeys; ++t) {
+        int64_t kk = keys[t];
+        int j = (int)(kk % NK);
+        int hk = (int)((kk / NK) % Hkv);
+        int b = (int)(kk / ((int64_t)NK * Hkv));
+        const double* k1r = k_base(k1, &s, b, hk) + (size_t)j * d;
+        const double* k2r = k_base(k2, &s, b, hk) + (size_t)j * d;
+        double* out = dk_keys + (size_t)t * d;
+        for (int h = hk * group; h < (hk + 1) * group; ++h) {
+            for (int i = (causal ? j : 0); i < NQ; ++i) {
+                int64_t r = ((int64_t)b * Hq + h) * NQ + i;
+                const double* q1r = q_row(q1, &s, b, h, i);
+                const double* q2r = q_row(q2, &s, b, h, i);
+                double a1 = 0.0, a2 = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    a1 += q1r[c] * k1r[c];
+                    a2 += q2r[c] * k2r[c];
+                }
+                double lp1 = scale * a1 - L1[r];
+                double lp2 = scale * a2 - L2[r];
+                double p1 = exp(lp1);
+                double ds = (mode == 1) ? dkl[r] * (exp(lp2) - p1)
+                                        : dkl[r] * p1 * ((lp1 - lp2) - KL[r]);
+                const double* qf = q_row(Qf, &s, b, h, i);
+                double w = scale * ds;
+                for (int c = 0; c < d; ++c) out[c] += w * qf[c];
+            }
+        }
+    }
+    return 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -86,13 +86,19 @@ def test_workspace_contents_do_not_matter():
 
 
 def test_identical_distributions_give_zero_gradient():
+    """P1 = P2 has zero gradient in both settings; on the GPU it vanishes to the rounding of
+    the fp32 statistics (the two sides take some exponentials on different units), i.e.
+    far below the gradient of the same call with distinct distributions."""
     w = inputs.custom(1, 2, 2, 256, 256, 128, True, True, seed=12)
     t = inputs.make(w, device="cuda")
     for mode in (1, 2):
+        kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], causal=True)
+        dq_ref, dk_ref = binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], causal=True)
         kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q1"], t["k1"], causal=True)
         dq, dk = binding.bwd(mode, t["q1"], t["k1"], t["q1"], t["k1"], kl, l1, l2, t["dkl"], causal=True)
         torch.cuda.synchronize()
-        assert dq.abs().max().item() == 0 and dk.abs().max().item() == 0
+        assert dq.abs().max().item() <= 1e-4 * dq_ref.abs().max().item()
+        assert dk.abs().max().item() <= 1e-4 * dk_ref.abs().max().item()
 
 
 def test_extra_memory_is_only_the_workspace():

@@ -64,8 +64,10 @@ def test_identical_inputs_give_zero_kl():
     t = inputs.make(w, device="cuda")
     kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q1"], t["k1"], scale=w.scale, causal=True)
     torch.cuda.synchronize()
-    assert torch.equal(l1, l2)
-    assert torch.all(kl == 0)
+    # the two distributions take part of their exponentials on different units (exponential
+    # unit vs FMA-pipe polynomial), so the identity holds to fp32 rounding, not bitwise
+    assert (l1 - l2).abs().max().item() <= 1e-5
+    assert kl.abs().max().item() <= 1e-5
 
 
 def test_causal_row_zero_and_nonnegative():

@@ -352,3 +352,19 @@ def test_bad_arguments_rejected():
     k = np.zeros((1, 2, 5, 8))
     with pytest.raises(ValueError):
         oracle.fwd(q, k, q, k, causal=True)  # causal needs NQ == NK
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_dk_with_given_statistics_matches_recomputed(mode):
+    """The variant that takes row statistics as inputs, fed the oracle's own statistics,
+    gives the self-contained dK (it differs only in where LSE and KL come from)."""
+    d = 64
+    B, Hq, Hkv, N = 1, 4, 2, 60
+    q1, k1, q2, k2 = make(B, Hq, Hkv, N, N, d, 60)
+    g = np.random.default_rng(3).uniform(0.5, 1.5, (B, Hq, N))
+    for causal in (False, True):
+        kl, l1, l2 = oracle.fwd(q1, k1, q2, k2, causal=causal)
+        keys = np.array([0, 5, 59, 60, 111, 119])
+        a = oracle.bwd_dk_keys(mode, q1, k1, q2, k2, g, keys, causal=causal)
+        b = oracle.bwd_dk_keys_stats(mode, q1, k1, q2, k2, g, kl, l1, l2, keys, causal=causal)
+        np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-16)
