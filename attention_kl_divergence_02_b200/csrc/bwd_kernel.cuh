@@ -13,24 +13,26 @@
 // on), so each (query tile, key tile) pair is visited exactly once ("Fusão de Kernel").
 // Per visit n:
 //   tensor core : S1 = Q1 K1^T, S2 = Q2 K2^T               (TMEM, lane = query row)
-//   4 warpgroups: dS for 32 key columns each (thread = query row, so the row's LSEs, KL
-//                 and g sit in registers) -> bf16, written once into a swizzled shared
-//                 tile [query][key] that serves both MMAs below
+//   4 compute warpgroups: dS for 32 key columns each (thread = query row, so the row's
+//                 LSEs, KL and g sit in registers) -> bf16, written once into a swizzled
+//                 shared tile [query][key] that serves both MMAs below
 //   tensor core : dK += dS^T Q_free   (dS read MN-major; TMEM accumulator over all
 //                                      visits, lane = key: no atomics)
 //                 dQp  = dS K_free    (dS read K-major; TMEM, lane = query row)
-//   4 warpgroups: dQp staged through shared memory and added into the fp32 dQ workspace
-//                 with bulk L2 reductions (cp.reduce.async.bulk .add.f32), off the L1 path
+//   flush warpgroup: dQp from TMEM through a double-buffered shared staging area into the
+//                 fp32 dQ workspace with bulk L2 reductions (cp.reduce.async.bulk .add.f32),
+//                 off the L1 path and off the compute warps' critical path
 // The workspace is private to the library and tile-blocked: one contiguous 128 x d block
-// per (batch, head, query tile), laid out in the order the warps hold it
-// ([warpgroup][lane quarter][4-column group][lane][4]), so that each warp's share is one
-// contiguous range; the convert kernel turns it into row-major bf16 dQ.
+// per (batch, head, query tile), laid out [lane quarter][32-column chunk][4-column group]
+// [lane][4], the order in which the flush warps hold it, so every 32-row x 32-column chunk
+// is one contiguous 4 KiB range; the convert kernel turns it into row-major bf16 dQ.
 // The MMA issuer looks one visit ahead: S of visit n+1 runs on the tensor core while the
-// warpgroups turn S of visit n into dS (needs two query stages in shared memory).
+// compute warpgroups turn S of visit n into dS (needs two query stages in shared memory).
 //
-// Roles (640 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
-// warps 2-3 idle, warps 4..19 = four 128-thread compute warpgroups (warp w touches TMEM
-// lanes 32*(w%4)..+31).
+// Roles (704 threads): warps 0-3 = dQ flush warpgroup, warps 4..19 = four compute
+// warpgroups, warp 20 = TMA producer, warp 21 = TMEM allocator + MMA issuer.  Warp w may
+// touch TMEM lanes 32*(w%4)..+31, which is why each 128-lane reader is a group of four
+// consecutive warps starting at a multiple of four.
 #pragma once
 
 #include "sm100.cuh"
@@ -49,12 +51,15 @@ struct BwdParams {
     const float* lse1;
     const float* lse2;
     const float* dkl;
-    float* dq_ws;   // fp32 [B,Hq,NQ,d]
+    float* dq_ws;   // fp32, tile-blocked (see above)
     uint16_t* dk;   // bf16 [B,Hkv,NK,d]
 };
 
-constexpr int kBwdThreads = 640;
-constexpr int kBwdWG = 4;   // compute warpgroups
+constexpr int kBwdThreads = 704;
+constexpr int kBwdWG = 4;          // compute warpgroups
+constexpr int kBwdComputeWarp0 = 4;
+constexpr int kBwdProducerWarp = 20;
+constexpr int kBwdMmaWarp = 21;
 
 template <int D, bool SHARED_K>
 struct BwdCfg {
@@ -65,10 +70,10 @@ struct BwdCfg {
     static constexpr int kNK = SHARED_K ? 1 : 2;                   // resident key tiles
     static constexpr int kK = 0;                                   // key tile i at kK + i*kTile
     static constexpr int kQ = kNK * kTile;                         // stage s: Q1 at kQ + s*2*kTile, Q2 after
-    static constexpr int kDS = kQ + kQS * 2 * kTile;               // dS^T tile, 128 x 128 bf16
-    static constexpr int kStage = kDS + 128 * 128 * 2;             // dQ staging, 2 KiB per compute warp
-    static constexpr int kStageWarp = 2048;
-    static constexpr int kBar = kStage + 4 * kBwdWG * kStageWarp;
+    static constexpr int kDS = kQ + kQS * 2 * kTile;               // dS tile, 128 x 128 bf16
+    static constexpr int kStage = kDS + 128 * 128 * 2;             // dQ staging: 4 warps x 2 x 4 KiB
+    static constexpr int kStageSlot = 4096;                        // 32 rows x 32 fp32 columns
+    static constexpr int kBar = kStage + 4 * 2 * kStageSlot;
     static constexpr int K_FULL = 0;
     static constexpr int Q_FULL = 1;                // + s
     static constexpr int Q_EMPTY = 1 + kQS;         // + s
@@ -121,11 +126,11 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, ui
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// This thread's bulk groups have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_all() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+// At most one of this thread's bulk groups is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_le1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
-// This thread's bulk groups have completed (global writes done).
+// All of this thread's bulk groups have completed (global writes done).
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -147,33 +152,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
-// D/4 columns of one TMEM lane (32 for d = 128, 16 for d = 64).
-template <int D>
-__device__ __forceinline__ void tmem_ld_quarter(uint32_t taddr, float (&v)[D / 4]) {
-    if constexpr (D == 128) {
-        uint32_t r[32];
-        tmem_ld32(taddr, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
-    } else {
-        uint32_t r[16];
-        tmem_ld16(taddr, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
-    }
-}
-
-// dS of one query row over 32 key columns, packed to bf16 pairs.  x = S1 raw, y = S2 raw;
+// dS of one query row over 16 key columns, packed to bf16 pairs.  x = S1 raw, y = S2 raw;
 // a = LSE1*log2(e); b = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2); g = upstream
 // gradient.  FOLDED: g >= 0 has been folded into the exponents (a and, in mode 1, b
 // lowered by log2 g, so 2^(u - a) is already g*P) and g is not multiplied again.  Adjacent
 // columns are processed as fp32x2 pairs.  With MASKED, columns k >= lim are zero.
 template <int MODE, bool MASKED, bool FOLDED>
-__device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
-                                         float sl2, float scale, float a, float b, float g,
-                                         int lim, uint32_t (&packed)[16]) {
+__device__ __forceinline__ void ds_half(const uint32_t (&xa)[16], const uint32_t (&ya)[16],
+                                        float sl2, float scale, float a, float b, float g,
+                                        int lim, uint32_t* packed) {
     const float2 sl = make_float2(sl2, sl2);
     const float2 na = make_float2(-a, -a);
     const float2 nb = make_float2(-b, -b);
@@ -182,7 +169,7 @@ __device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[32], const uint32_
     const float2 sc = make_float2(scale, scale);
     const float2 neg1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int pr = 0; pr < 16; ++pr) {
+    for (int pr = 0; pr < 8; ++pr) {
         const float2 xk = make_float2(__uint_as_float(xa[2 * pr]), __uint_as_float(xa[2 * pr + 1]));
         const float2 yk = make_float2(__uint_as_float(ya[2 * pr]), __uint_as_float(ya[2 * pr + 1]));
         const float2 u1 = __ffma2_rn(xk, sl, na);
@@ -203,6 +190,19 @@ __device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[32], const uint32_
             if (2 * pr + 1 >= lim) v.y = 0.f;
         }
         packed[pr] = pack_bf16(v.x, v.y);
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void ds_half_any(bool masked, bool folded, const uint32_t (&xa)[16],
+                                            const uint32_t (&ya)[16], float sl2, float scale,
+                                            float a, float b, float g, int lim, uint32_t* packed) {
+    if (folded) {
+        if (masked) ds_half<MODE, true, true>(xa, ya, sl2, scale, a, b, g, lim, packed);
+        else ds_half<MODE, false, true>(xa, ya, sl2, scale, a, b, g, 16, packed);
+    } else {
+        if (masked) ds_half<MODE, true, false>(xa, ya, sl2, scale, a, b, g, lim, packed);
+        else ds_half<MODE, false, false>(xa, ya, sl2, scale, a, b, g, 16, packed);
     }
 }
 
@@ -248,13 +248,13 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         mbar_init(BAR(C::DS_FULL), 32 * 4 * kBwdWG);
         mbar_init(BAR(C::DS_FREE), 1);
         mbar_init(BAR(C::DQ_FULL), 1);
-        mbar_init(BAR(C::DQ_FREE), 32 * 4 * kBwdWG);
+        mbar_init(BAR(C::DQ_FREE), 128);
         mbar_init(BAR(C::DK_FULL), 1);
         mbar_init(BAR(C::DONE), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kBwdMmaWarp) {
         tmem_alloc(smem_u32(tmem_holder), 512);
         tmem_relinquish();
     }
@@ -263,7 +263,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0) {
+    if (warp == kBwdProducerWarp) {
         // ================================================================ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ1);
@@ -302,7 +302,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kBwdMmaWarp) {
         // ================================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // Q, K both K-major
@@ -382,55 +382,65 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             mma_commit(BAR(C::DONE));
             drain_wait(BAR(C::DONE), 0);
         }
-    } else if (warp >= 4) {
+    } else if (warp < kBwdComputeWarp0) {
+        // ================================================================ dQ flush warpgroup
+        const int quarter = warp;               // TMEM lanes 32*quarter.. = query rows
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        // this warp's two 4 KiB staging slots, each [4-column group (8)][lane (32)][4 floats]
+        float4* slots = reinterpret_cast<float4*>(smem + C::kStage + warp * 2 * C::kStageSlot);
+        const uint32_t slots_s = smem_u32(slots);
+        int chunk = 0;                          // running chunk count: slot = chunk & 1
+        for (int n = 0; n < N; ++n) {
+            int h, qt;
+            sched.visit(n, h, qt);
+            if (!mbar_wait(BAR(C::DQ_FULL), n & 1, abort_flag)) break;
+            tc_fence_after();
+            float* blk = p.dq_ws + ((size_t)(b * p.Hq + h) * p.nqt + qt) * (128 * D) +
+                         (size_t)quarter * (32 * D);
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c, ++chunk) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + C::kColDQ + c * 32, v);
+                tmem_wait_ld();
+                if (c == D / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(BAR(C::DQ_FREE));   // the dQ columns are all in registers
+                }
+                float4* slot = slots + (chunk & 1) * (C::kStageSlot / 16);
+                if (lane == 0) bulk_wait_read_le1();   // the slot's previous chunk was read
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    slot[g * 32 + lane] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                                      __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_reduce_add_f32(blk + c * (32 * 32), slots_s + (chunk & 1) * C::kStageSlot,
+                                        C::kStageSlot);
+                    bulk_commit();
+                }
+            }
+        }
+        // every bulk reduction this warp started has landed before the CTA exits
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    } else if (warp < kBwdComputeWarp0 + 4 * kBwdWG) {
         // ================================================================ compute warpgroups
-        const int wg = (warp - 4) >> 2;         // key columns [32*wg, 32*wg + 32)
+        const int wg = (warp - kBwdComputeWarp0) >> 2;   // key columns [32*wg, 32*wg + 32)
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;      // TMEM lane: query row (S, dQ) or key row (dK)
+        const int r = quarter * 32 + lane;      // TMEM lane: query row (S) or key row (dK)
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.sl2;
         const float scale = p.scale;
         const float LOG2E = 1.4426950408889634f;
         uint8_t* ds_tile = smem + C::kDS;
-        // this thread's 64 bytes of the dS^T row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
+        // this thread's 64 bytes of dS row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
         uint8_t* ds_row = ds_tile + (wg >> 1) * C::kBox + r * 128;
-        // this warp's dQ staging slot: [4-column group (4)][lane (32)][4 floats] = 2 KiB
-        float4* stage = reinterpret_cast<float4*>(smem + C::kStage + (warp - 4) * C::kStageWarp);
-        const uint32_t stage_s = smem_u32(stage);
-        constexpr int kCols = D / 4;          // dQ / dK columns per warpgroup
-        constexpr int kRounds = D / 64;       // 2 KiB staging rounds per visit
         bool ok = true;
-        int prev_bh = 0, prev_qt = 0;
-        // Move this warp's share of the dQ partial of an earlier visit into the workspace
-        // block of (bh_, qt_): TMEM -> registers -> staging slot -> bulk L2 reduction.
-        auto flush_dq = [&](int n_done, int bh_, int qt_) -> bool {
-            if (!mbar_wait(BAR(C::DQ_FULL), n_done & 1, abort_flag)) return false;
-            tc_fence_after();
-            float v[kCols];
-            tmem_ld_quarter<D>(lane_base + C::kColDQ + wg * kCols, v);
-            tc_fence_before();
-            mbar_arrive(BAR(C::DQ_FREE));
-            float* blk = p.dq_ws + ((size_t)bh_ * p.nqt + qt_) * (128 * D) +
-                         (size_t)(wg * 4 + quarter) * (32 * kCols);
-#pragma unroll
-            for (int rd = 0; rd < kRounds; ++rd) {
-                if (lane == 0) bulk_wait_read_all();   // the slot's previous contents were read
-                __syncwarp();
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int c = (rd * 4 + g) * 4;
-                    stage[g * 32 + lane] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    bulk_reduce_add_f32(blk + rd * 512, stage_s, C::kStageWarp);
-                    bulk_commit();
-                }
-            }
-            return true;
-        };
-        // per-row statistics of visit n for this thread's query row
+        // per-row statistics of visit n for this thread's query row: ra = LSE1*log2(e),
+        // rb = LSE2*log2(e) (mode 1) or LSE2 - LSE1 - KL (mode 2), rg = g; rows past NQ
+        // get g = 0 (their dS is 0)
         auto load_row_consts = [&](int n, float& ra, float& rb, float& rg) {
             int h, qt;
             sched.visit(n, h, qt);
@@ -451,49 +461,48 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         for (int n = 0; n < N; ++n) {
             int h, qt;
             sched.visit(n, h, qt);
-            const int bh = b * p.Hq + h;
-            const int q0 = qt * 128;
-            // this thread's query row: ca = LSE1*log2(e), cb = LSE2*log2(e) (mode 1) or
-            // LSE2 - LSE1 - KL (mode 2), cg = g; rows past NQ get g = 0 (their dS is 0).
-            // The next visit's values are loaded now and used one iteration later.
+            // this visit's statistics were loaded one iteration ago; start the next ones
             const float ca = na, cb = nb, cg = ng;
             if (n + 1 < N) load_row_consts(n + 1, na, nb, ng);
+            // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf
+            // makes a row with g = 0 give exactly 0)
+            const bool folded = !__any_sync(0xffffffffu, cg < 0.f);
+            float a = ca, bq = cb;
+            if (folded) {
+                const float lg = log2f(cg);
+                a = ca - lg;
+                if (mode1) bq = cb - lg;
+            }
+            // masked columns: keys past the diagonal of a causal diagonal tile, and
+            // zero-filled keys past NK; columns k < lim of this warpgroup are valid
+            const int kc0 = wg * 32;
+            const bool need_mask = (p.causal && qt == kt) || (k0 + 128 > p.NK);
+            int lim = 32;
+            if (need_mask) {
+                lim = min(lim, p.NK - k0 - kc0);
+                if (p.causal && qt == kt) lim = min(lim, r - kc0 + 1);
+            }
             if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t xa[32], ya[32];
-            tmem_ld32(lane_base + C::kColS1 + wg * 32, xa);
-            tmem_ld32(lane_base + C::kColS2 + wg * 32, ya);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(BAR(C::S_FREE));
-            // dS[r, key] for the 32 key columns.  Masked: keys past the diagonal of a causal
-            // diagonal tile and zero-filled keys past NK.
-            const int kc0 = wg * 32;               // first key column of this warpgroup
-            const bool need_mask = (p.causal && qt == kt) || (k0 + 128 > p.NK);
-            int lim = 32;                          // columns k < lim are valid keys
-            if (need_mask) {
-                lim = min(lim, p.NK - k0 - kc0);
-                if (p.causal && qt == kt) lim = min(lim, r - kc0 + 1);
-            }
             uint32_t packed[16];
-            // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf
-            // makes a row with g = 0 give exactly 0)
-            if (!__any_sync(0xffffffffu, cg < 0.f)) {
-                const float lg = log2f(cg);
-                const float fa = ca - lg;
-                const float fb = mode1 ? cb - lg : cb;
-                if (need_mask)
-                    ds_chunk<MODE, true, true>(xa, ya, sl2, scale, fa, fb, cg, lim, packed);
-                else
-                    ds_chunk<MODE, false, true>(xa, ya, sl2, scale, fa, fb, cg, 32, packed);
-            } else {
-                if (need_mask)
-                    ds_chunk<MODE, true, false>(xa, ya, sl2, scale, ca, cb, cg, lim, packed);
-                else
-                    ds_chunk<MODE, false, false>(xa, ya, sl2, scale, ca, cb, cg, 32, packed);
+            {
+                uint32_t xa[16], ya[16];
+                tmem_ld16(lane_base + C::kColS1 + kc0, xa);
+                tmem_ld16(lane_base + C::kColS2 + kc0, ya);
+                tmem_wait_ld();
+                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, cg, lim, packed);
+            }
+            {
+                uint32_t xa[16], ya[16];
+                tmem_ld16(lane_base + C::kColS1 + kc0 + 16, xa);
+                tmem_ld16(lane_base + C::kColS2 + kc0 + 16, ya);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(BAR(C::S_FREE));      // all of this thread's S columns are read
+                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, cg, lim - 16, packed + 8);
             }
             if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
                 ok = false;
@@ -508,36 +517,34 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             }
             fence_async_smem();
             mbar_arrive(BAR(C::DS_FULL));
-            if (n > 0 && !flush_dq(n - 1, prev_bh, prev_qt)) {
-                ok = false;
-                break;
-            }
-            prev_bh = bh;
-            prev_qt = qt;
         }
-        if (ok && N > 0) ok = flush_dq(N - 1, prev_bh, prev_qt);
         if (ok && mbar_wait(BAR(C::DK_FULL), 0, abort_flag)) {
             tc_fence_after();
-            float v[kCols];
-            tmem_ld_quarter<D>(lane_base + C::kColDK + wg * kCols, v);
+            constexpr int kCols = D / 4;          // dK columns per warpgroup
+            uint32_t v[kCols];
+            if constexpr (D == 128) {
+                tmem_ld32(lane_base + C::kColDK + wg * kCols, v);
+            } else {
+                tmem_ld16(lane_base + C::kColDK + wg * kCols, v);
+            }
+            tmem_wait_ld();
             if (k0 + r < p.NK) {
                 uint4* dst = reinterpret_cast<uint4*>(p.dk + ((size_t)bhk * p.NK + k0 + r) * D + wg * kCols);
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    dst[k] = make_uint4(pack_bf16(v[8 * k] * scale, v[8 * k + 1] * scale),
-                                        pack_bf16(v[8 * k + 2] * scale, v[8 * k + 3] * scale),
-                                        pack_bf16(v[8 * k + 4] * scale, v[8 * k + 5] * scale),
-                                        pack_bf16(v[8 * k + 6] * scale, v[8 * k + 7] * scale));
+                for (int k = 0; k < kCols / 8; ++k) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * k + e]) * scale;
+                    dst[k] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]),
+                                        pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+                }
             }
         }
-        // every bulk reduction this warp started has landed before the CTA exits
-        if (lane == 0) bulk_wait_all();
-        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kBwdMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -545,33 +552,34 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 }
 
 // dq = bf16(scale * ws), un-blocking the tile-blocked workspace.  One thread = one query
-// row's D/4 columns of one warpgroup slice: it reads D/16 float4 (coalesced across the 32
-// lanes of the block) and writes D/2 contiguous bytes of its dQ row.
+// row's 32-column chunk: it reads 8 float4 (coalesced across the 32 lanes of the chunk) and
+// writes 64 contiguous bytes of its dQ row.
 template <int D>
 __global__ void __launch_bounds__(256)
 streamkl_dq_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dq, int BH, int NQ,
                            int nqt, float scale) {
-    constexpr int kCols = D / 4;
-    const size_t total = (size_t)BH * nqt * 512;   // (bh, tile, wg, quarter, lane)
+    constexpr int kChunks = D / 32;
+    const size_t total = (size_t)BH * nqt * 128 * kChunks;   // (bh, tile, quarter, chunk, lane)
     for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
          t += (size_t)gridDim.x * blockDim.x) {
         const int lane = (int)(t & 31);
-        const int quarter = (int)((t >> 5) & 3);
-        const int wg = (int)((t >> 7) & 3);
-        const size_t blk = t >> 9;                 // bh * nqt + qt
+        const size_t u = t >> 5;
+        const int c = (int)(u % kChunks);
+        const int quarter = (int)((u / kChunks) & 3);
+        const size_t blk = u / kChunks / 4;        // bh * nqt + qt
         const int qt = (int)(blk % nqt);
         const size_t bh = blk / nqt;
         const int q = qt * 128 + quarter * 32 + lane;
         if (q >= NQ) continue;
         const float4* src = reinterpret_cast<const float4*>(
-            ws + blk * (128 * D) + (size_t)(wg * 4 + quarter) * (32 * kCols)) + lane;
-        uint4* dst = reinterpret_cast<uint4*>(dq + (bh * NQ + q) * D + wg * kCols);
+            ws + blk * (128 * D) + (size_t)(quarter * kChunks + c) * 1024) + lane;
+        uint4* dst = reinterpret_cast<uint4*>(dq + (bh * NQ + q) * D + c * 32);
 #pragma unroll
-        for (int k = 0; k < kCols / 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
             const float4 a = src[(2 * k) * 32];
-            const float4 c = src[(2 * k + 1) * 32];
+            const float4 e = src[(2 * k + 1) * 32];
             dst[k] = make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
-                                pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+                                pack_bf16(e.x * scale, e.y * scale), pack_bf16(e.z * scale, e.w * scale));
         }
     }
 }

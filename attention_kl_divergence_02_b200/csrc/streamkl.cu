@@ -110,7 +110,7 @@ int launch_bwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
     kern<<<grid, skl::kBwdThreads, smem, st>>>(q1, q2, k1, k2, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_bwd launch");
-    const size_t threads = (size_t)p.B * p.Hq * p.nqt * 512;
+    const size_t threads = (size_t)p.B * p.Hq * p.nqt * 128 * (D / 32);
     size_t blocks = (threads + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
     skl::streamkl_dq_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(p.dq_ws, dq, p.B * p.Hq,
