@@ -64,7 +64,7 @@ def load(path=None):
     lib.streamkl_bwd_noalloc.argtypes = ([i, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
                                           vp, vp, vp])
     lib.streamkl_bwd_noalloc.restype = i
-    lib.streamkl_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.streamkl_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.streamkl_bwd_workspace_bytes.restype = sz
     lib.streamkl_status_string.argtypes = [i]
     lib.streamkl_status_string.restype = ctypes.c_char_p
@@ -118,7 +118,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 def streamkl_bwd_noalloc(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
                          causal, dq, dk, stream=None):
     """Backward without a workspace argument, for callers that may not allocate device
-    memory: the library's fixed 32 MiB built-in buffer holds the dQ accumulator.  Calls
+    memory: the library's fixed 32 MiB built-in buffer holds the dK accumulator.  Calls
     that can overlap on the GPU share that buffer and race; larger problems return
     ERR_UNSUPPORTED."""
     return load().streamkl_bwd_noalloc(int(mode), _ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(kl),
@@ -127,8 +127,8 @@ def streamkl_bwd_noalloc(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, 
                                        _stream(stream))
 
 
-def streamkl_bwd_workspace_bytes(B, Hq, NQ, d):
-    return load().streamkl_bwd_workspace_bytes(B, Hq, NQ, d)
+def streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d):
+    return load().streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d)
 
 
 def streamkl_device_status(stream=None):
@@ -186,7 +186,7 @@ def bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, scale=None, causal=False, out
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if out is None:
         out = (torch.empty_like(q1), torch.empty_like(k1))
-    nbytes = streamkl_bwd_workspace_bytes(B, Hq, NQ, d)
+    nbytes = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16) // 4, dtype=torch.float32, device=q1.device)
     rc = streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,

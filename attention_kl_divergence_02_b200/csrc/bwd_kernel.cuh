@@ -8,28 +8,30 @@
 // and the mode-2 log-ratio taken from logit differences, never log P ("Estabilidade
 // Numérica").  dQ = scale * dS K, dK = scale * dS^T Q.
 //
-// One CTA owns one 128-key tile of one (batch, KV head) and visits every 128-row query
-// tile of every query head in the KV group that can see it (causal: from the diagonal
-// on), so each (query tile, key tile) pair is visited exactly once ("Fusão de Kernel").
-// Per visit n:
+// One CTA owns one 128-row query tile of one (batch, query head): Q1, Q2 and the rows'
+// saved statistics stay on chip while the key tiles the rows can see (causal: up to the
+// diagonal) stream through a ring of shared-memory slots, so each (query tile, key tile)
+// pair is visited exactly once ("Fusão de Kernel").  Per visit n:
 //   tensor core : S1 = Q1 K1^T, S2 = Q2 K2^T               (TMEM, lane = query row)
-//   4 compute warpgroups: dS for 32 key columns each (thread = query row, so the row's
-//                 LSEs, KL and g sit in registers) -> bf16, written once into a swizzled
-//                 shared tile [query][key] that serves both MMAs below
-//   tensor core : dK += dS^T Q_free   (dS read MN-major; TMEM accumulator over all
-//                                      visits, lane = key: no atomics)
-//                 dQp  = dS K_free    (dS read K-major; TMEM, lane = query row)
-//   flush warpgroup: dQp from TMEM through a double-buffered shared staging area into the
-//                 fp32 dQ workspace with bulk L2 reductions (cp.reduce.async.bulk .add.f32),
-//                 off the L1 path and off the compute warps' critical path
-// The workspace is private to the library and tile-blocked: one contiguous 128 x d block
-// per (batch, head, query tile), laid out [lane quarter][32-column chunk][4-column group]
-// [lane][4], the order in which the flush warps hold it, so every 32-row x 32-column chunk
-// is one contiguous 4 KiB range; the convert kernel turns it into row-major bf16 dQ.
-// The MMA issuer looks one visit ahead: S of visit n+1 runs on the tensor core while the
-// compute warpgroups turn S of visit n into dS (needs two query stages in shared memory).
+//   4 compute warpgroups: dS for 32 key columns each (thread = query row: the row's LSEs,
+//                 KL and g sit in registers for the CTA's whole life) -> bf16, written
+//                 once into a swizzled shared tile [query][key] that feeds both MMAs below
+//   tensor core : dQ += dS K_free    (dS read K-major; TMEM accumulator over all visits:
+//                                     dQ never leaves the chip until the end)
+//                 dKp  = dS^T Q_free (dS read MN-major; TMEM, lane = key)
+//   flush warpgroup: dKp from TMEM through a double-buffered shared staging area into an
+//                 fp32 dK workspace with bulk L2 reductions (cp.reduce.async.bulk .add.f32)
+// Streaming the key tile (32 KiB with shared keys) instead of the query pair keeps the
+// per-visit load small enough for a ring that prefetches two visits ahead, and the MMA
+// issuer looks one visit ahead: S of visit n+1 runs while the warpgroups turn S of visit n
+// into dS.
 //
-// Roles (704 threads): warps 0-3 = dQ flush warpgroup, warps 4..19 = four compute
+// The workspace is private to the library and tile-blocked: one contiguous 128 x d block
+// per (batch, KV head, key tile), laid out [lane quarter][32-column chunk][4-column group]
+// [lane][4], the order in which the flush warps hold it; the convert kernel turns it into
+// row-major bf16 dK.
+//
+// Roles (704 threads): warps 0-3 = dK flush warpgroup, warps 4..19 = four compute
 // warpgroups, warp 20 = TMA producer, warp 21 = TMEM allocator + MMA issuer.  Warp w may
 // touch TMEM lanes 32*(w%4)..+31, which is why each 128-lane reader is a group of four
 // consecutive warps starting at a multiple of four.
@@ -42,7 +44,6 @@ namespace skl {
 struct BwdParams {
     int B, Hq, Hkv, NQ, NK;
     int causal;
-    int mode;
     int nkt;        // key tiles per (b, KV head)
     int nqt;        // query tiles per head
     float sl2;      // scale * log2(e)
@@ -51,8 +52,8 @@ struct BwdParams {
     const float* lse1;
     const float* lse2;
     const float* dkl;
-    float* dq_ws;   // fp32, tile-blocked (see above)
-    uint16_t* dk;   // bf16 [B,Hkv,NK,d]
+    float* dk_ws;   // fp32, tile-blocked (see above)
+    uint16_t* dq;   // bf16 [B,Hq,NQ,d]
 };
 
 constexpr int kBwdThreads = 704;
@@ -63,57 +64,51 @@ constexpr int kBwdMmaWarp = 21;
 
 template <int D, bool SHARED_K>
 struct BwdCfg {
-    static constexpr int kTile = 128 * D * 2;
+    static constexpr int kTile = 128 * D * 2;                      // one 128-row bf16 tile
     static constexpr int kBoxes = D / 64;
     static constexpr int kBox = 128 * 128;
-    static constexpr int kQS = (D == 128 && !SHARED_K) ? 1 : 2;   // query stages
-    static constexpr int kNK = SHARED_K ? 1 : 2;                   // resident key tiles
-    static constexpr int kK = 0;                                   // key tile i at kK + i*kTile
-    static constexpr int kQ = kNK * kTile;                         // stage s: Q1 at kQ + s*2*kTile, Q2 after
-    static constexpr int kDS = kQ + kQS * 2 * kTile;               // dS tile, 128 x 128 bf16
-    static constexpr int kStage = kDS + 128 * 128 * 2;             // dQ staging: 4 warps x 2 x 4 KiB
+    static constexpr int kPerVisit = SHARED_K ? 1 : 2;             // key tiles streamed per visit
+    static constexpr int kSlots = (D == 128) ? 3 : 8;              // key-tile ring
+    static constexpr int kQ1 = 0;
+    static constexpr int kQ2 = kTile;
+    static constexpr int kRing = 2 * kTile;                        // slot s at kRing + s*kTile
+    static constexpr int kDS = kRing + kSlots * kTile;             // dS tile, 128 x 128 bf16
+    static constexpr int kStage = kDS + 128 * 128 * 2;             // dK staging: 4 warps x 2 x 4 KiB
     static constexpr int kStageSlot = 4096;                        // 32 rows x 32 fp32 columns
     static constexpr int kBar = kStage + 4 * 2 * kStageSlot;
-    static constexpr int K_FULL = 0;
-    static constexpr int Q_FULL = 1;                // + s
-    static constexpr int Q_EMPTY = 1 + kQS;         // + s
-    static constexpr int S_FULL = 1 + 2 * kQS;
+    static constexpr int Q_FULL = 0;
+    static constexpr int K_FULL = 1;                // + s
+    static constexpr int K_EMPTY = 1 + kSlots;      // + s
+    static constexpr int S_FULL = 1 + 2 * kSlots;
     static constexpr int S_FREE = S_FULL + 1;
     static constexpr int DS_FULL = S_FULL + 2;
     static constexpr int DS_FREE = S_FULL + 3;
-    static constexpr int DQ_FULL = S_FULL + 4;
-    static constexpr int DQ_FREE = S_FULL + 5;
-    static constexpr int DK_FULL = S_FULL + 6;
+    static constexpr int DK_FULL = S_FULL + 4;
+    static constexpr int DK_FREE = S_FULL + 5;
+    static constexpr int DQ_DONE = S_FULL + 6;
     static constexpr int DONE = S_FULL + 7;
     static constexpr int kNumBars = DONE + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kSmem = kMisc + 16 + 1024;
-    static constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDK = 256, kColDQ = 384;
+    static constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDQ = 256, kColDK = 384;
 };
 
-// Visit n of a CTA -> (query head, query tile).  Causal: every head of the group, query
-// tiles from the diagonal on.  Non-causal: all (head, tile) pairs, rotated by the key tile
-// index so that CTAs of one head start on different dQ rows.
+// Visit n of a CTA -> key tile.  Causal: key tiles qt, qt-1, ..., 0 (diagonal first).
+// Non-causal: all key tiles, rotated by query tile and head so that CTAs working at the
+// same time reduce into different dK blocks.
 struct BwdSchedule {
-    int hk0, G, nqt, kt, causal, count;
-    __device__ BwdSchedule(const BwdParams& p, int hk, int kt_) {
-        G = p.Hq / p.Hkv;
-        hk0 = hk * G;
-        nqt = p.nqt;
-        kt = kt_;
+    int nkt, qt, rot, causal, count;
+    __device__ BwdSchedule(const BwdParams& p, int qt_, int h) {
+        nkt = p.nkt;
+        qt = qt_;
         causal = p.causal;
-        count = causal ? G * (nqt - kt) : G * nqt;
+        rot = (qt_ + h) % p.nkt;
+        count = causal ? qt_ + 1 : p.nkt;
     }
-    __device__ void visit(int n, int& h, int& qt) const {
-        if (causal) {
-            const int per = nqt - kt;
-            h = hk0 + n / per;
-            qt = kt + n % per;
-        } else {
-            const int u = (n + kt) % count;
-            h = hk0 + u / nqt;
-            qt = u % nqt;
-        }
+    __device__ int key_tile(int n) const {
+        if (causal) return qt - n;
+        const int u = n + rot;
+        return u >= nkt ? u - nkt : u;
     }
 };
 
@@ -224,32 +219,42 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    const int BHk = p.B * p.Hkv;
-    const int kt = blockIdx.x / BHk;     // key tile; kt = 0 (most visits when causal) first
-    const int bhk = blockIdx.x % BHk;
-    const int b = bhk / p.Hkv;
-    const int hk = bhk % p.Hkv;
-    const int k0 = kt * 128;
-    const BwdSchedule sched(p, hk, kt);
+    // ---- work unit: heaviest causal query tiles are handed out first
+    const int BH = p.B * p.Hq;
+    const int unit = blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
+    const int qt = p.causal ? (p.nqt - 1 - unit) : unit;
+    const int b = bh / p.Hq;
+    const int h = bh % p.Hq;
+    const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
+    const int q0 = qt * 128;
+    const BwdSchedule sched(p, qt, h);
     const int N = sched.count;
     constexpr bool mode1 = (MODE == 1);
-    // the free distribution's operands: mode 1 -> (Q2, K2), mode 2 -> (Q1, K1)
-    const uint32_t kfree = sb + C::kK + ((SHARED_K || !mode1) ? 0 : C::kTile);
-    const uint32_t k2tile = sb + C::kK + (SHARED_K ? 0 : C::kTile);
+    // Key tiles of a visit enter the ring in the order (fixed distribution's, free
+    // distribution's): j = 0 is released as soon as S is done, j = 1 after dQ.  With three
+    // slots, the look-ahead S(n+1) then lands in slots that S(n) and dQ(n-1) have freed.
+    // (With shared keys there is one tile per visit, j = 0, released after dQ.)
+    auto ring_idx = [](int n, int j) { return n * C::kPerVisit + j; };
+    // j of K1 and of K2; the free distribution is (Q2, K2) in mode 1, (Q1, K1) in mode 2
+    constexpr int kJ1 = SHARED_K ? 0 : (mode1 ? 0 : 1);
+    constexpr int kJ2 = SHARED_K ? 0 : (mode1 ? 1 : 0);
+    constexpr int kJFree = SHARED_K ? 0 : 1;
+    const uint32_t qfree = sb + (mode1 ? C::kQ2 : C::kQ1);
 
     if (threadIdx.x == 0) {
-        mbar_init(BAR(C::K_FULL), 1);
-        for (int s = 0; s < C::kQS; ++s) {
-            mbar_init(BAR(C::Q_FULL + s), 1);
-            mbar_init(BAR(C::Q_EMPTY + s), 1);
+        mbar_init(BAR(C::Q_FULL), 1);
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(BAR(C::K_FULL + s), 1);
+            mbar_init(BAR(C::K_EMPTY + s), 1);
         }
         mbar_init(BAR(C::S_FULL), 1);
         mbar_init(BAR(C::S_FREE), 32 * 4 * kBwdWG);
         mbar_init(BAR(C::DS_FULL), 32 * 4 * kBwdWG);
         mbar_init(BAR(C::DS_FREE), 1);
-        mbar_init(BAR(C::DQ_FULL), 1);
-        mbar_init(BAR(C::DQ_FREE), 128);
         mbar_init(BAR(C::DK_FULL), 1);
+        mbar_init(BAR(C::DK_FREE), 128);
+        mbar_init(BAR(C::DQ_DONE), 1);
         mbar_init(BAR(C::DONE), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -270,35 +275,37 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             tma_prefetch_desc(&tmQ2);
             tma_prefetch_desc(&tmK1);
             if (!SHARED_K) tma_prefetch_desc(&tmK2);
-            mbar_arrive_expect_tx(BAR(C::K_FULL), C::kNK * C::kTile);
+            mbar_arrive_expect_tx(BAR(C::Q_FULL), 2 * C::kTile);
             for (int bx = 0; bx < C::kBoxes; ++bx) {
-                tma_load_3d(sb + C::kK + bx * C::kBox, &tmK1, BAR(C::K_FULL), bx * 64, k0, bhk);
-                if (!SHARED_K)
-                    tma_load_3d(sb + C::kK + C::kTile + bx * C::kBox, &tmK2, BAR(C::K_FULL), bx * 64,
-                                k0, bhk);
+                tma_load_3d(sb + C::kQ1 + bx * C::kBox, &tmQ1, BAR(C::Q_FULL), bx * 64, q0, bh);
+                tma_load_3d(sb + C::kQ2 + bx * C::kBox, &tmQ2, BAR(C::Q_FULL), bx * 64, q0, bh);
             }
-            int n = 0;
-            for (; n < N; ++n) {
-                const int s = n % C::kQS;
-                const int u = n / C::kQS;
-                if (u > 0 && !mbar_wait(BAR(C::Q_EMPTY + s), (u - 1) & 1, abort_flag)) break;
-                int h, qt;
-                sched.visit(n, h, qt);
-                const int bh = b * p.Hq + h;
-                const uint32_t q1s = sb + C::kQ + s * 2 * C::kTile;
-                const uint32_t q2s = q1s + C::kTile;
-                mbar_arrive_expect_tx(BAR(C::Q_FULL + s), 2 * C::kTile);
-                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                    tma_load_3d(q1s + bx * C::kBox, &tmQ1, BAR(C::Q_FULL + s), bx * 64, qt * 128, bh);
-                    tma_load_3d(q2s + bx * C::kBox, &tmQ2, BAR(C::Q_FULL + s), bx * 64, qt * 128, bh);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int n = 0; n < N && ok; ++n) {
+                const int kt = sched.key_tile(n);
+#pragma unroll
+                for (int j = 0; j < C::kPerVisit; ++j) {
+                    const uint32_t s = it % C::kSlots;
+                    const uint32_t u = it / C::kSlots;
+                    if (u > 0 && !mbar_wait(BAR(C::K_EMPTY + s), (u - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(BAR(C::K_FULL + s), C::kTile);
+                    const CUtensorMap* map = (j == kJ1) ? &tmK1 : &tmK2;
+                    for (int bx = 0; bx < C::kBoxes; ++bx)
+                        tma_load_3d(sb + C::kRing + s * C::kTile + bx * C::kBox, map,
+                                    BAR(C::K_FULL + s), bx * 64, kt * 128, bhk);
+                    ++it;
                 }
             }
             // drain every copy started here
-            drain_wait(BAR(C::K_FULL), 0);
-            for (int s = 0; s < C::kQS; ++s) {
-                if (n > s) {
-                    const int fills = (n - s - 1) / C::kQS + 1;
-                    drain_wait(BAR(C::Q_FULL + s), (fills - 1) & 1);
+            drain_wait(BAR(C::Q_FULL), 0);
+            for (uint32_t s = 0; s < (uint32_t)C::kSlots; ++s) {
+                if (it > s) {
+                    const uint32_t fills = (it - s - 1) / C::kSlots + 1;
+                    drain_wait(BAR(C::K_FULL + s), (fills - 1) & 1);
                 }
             }
         }
@@ -306,105 +313,96 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         // ================================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // Q, K both K-major
-            constexpr uint32_t idK = idesc_bf16(128, D, 1, 1);     // dS^T MN-major, Q MN-major
             constexpr uint32_t idQ = idesc_bf16(128, D, 0, 1);     // dS K-major, K MN-major
-            auto issue_S = [&](int n) {
-                const int s = n % C::kQS;
-                const uint32_t q1s = sb + C::kQ + s * 2 * C::kTile;
-                const uint32_t q2s = q1s + C::kTile;
+            constexpr uint32_t idK = idesc_bf16(128, D, 1, 1);     // dS^T MN-major, Q MN-major
+            auto slot_of = [&](int n, int j) { return (uint32_t)(ring_idx(n, j) % C::kSlots); };
+            auto fill_parity = [&](int n, int j) { return (uint32_t)((ring_idx(n, j) / C::kSlots) & 1); };
+            // S of visit n; returns false if a wait gave up
+            auto issue_S = [&](int n) -> bool {
+                const uint32_t s1 = slot_of(n, kJ1);
+                if (!mbar_wait(BAR(C::K_FULL + s1), fill_parity(n, kJ1), abort_flag)) return false;
+                uint32_t s2 = s1;
+                if (!SHARED_K) {
+                    s2 = slot_of(n, kJ2);
+                    if (!mbar_wait(BAR(C::K_FULL + s2), fill_parity(n, kJ2), abort_flag)) return false;
+                }
+                tc_fence_after();
+                const uint32_t k1s = sb + C::kRing + s1 * C::kTile;
+                const uint32_t k2s = sb + C::kRing + s2 * C::kTile;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(q1s + off, 16, 1024),
-                                sw128_desc(sb + C::kK + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(sb + C::kQ1 + off, 16, 1024),
+                                sw128_desc(k1s + off, 16, 1024), idS, k > 0);
                 }
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(q2s + off, 16, 1024),
-                                sw128_desc(k2tile + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(sb + C::kQ2 + off, 16, 1024),
+                                sw128_desc(k2s + off, 16, 1024), idS, k > 0);
                 }
                 mma_commit(BAR(C::S_FULL));
+                // with distinct keys, the fixed distribution's key tile (j = 0) is done after S
+                if (!SHARED_K) mma_commit(BAR(C::K_EMPTY + slot_of(n, 0)));
+                return true;
             };
-            auto issue_dK = [&](int n) {
-                const int s = n % C::kQS;
-                const uint32_t qf = sb + C::kQ + s * 2 * C::kTile + (mode1 ? C::kTile : 0);
+            bool ok = mbar_wait(BAR(C::Q_FULL), 0, abort_flag);
+            if (ok) ok = issue_S(0);
+            for (int n = 0; n < N && ok; ++n) {
+                if (n + 1 < N) {
+                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+                    tc_fence_after();
+                    if (!issue_S(n + 1)) break;
+                }
+                if (!mbar_wait(BAR(C::DS_FULL), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (n > 0) {
+                    if (!mbar_wait(BAR(C::DK_FREE), (n - 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                }
+                // dK partial of this key tile: dS^T Q_free (fresh every visit)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
                     mma_bf16_ss(tmem + C::kColDK, sw128_desc(sb + C::kDS + k * 2048, C::kBox, 1024),
-                                sw128_desc(qf + k * 2048, C::kBox, 1024), idK, (n > 0 || k > 0));
+                                sw128_desc(qfree + k * 2048, C::kBox, 1024), idK, k > 0);
                 }
-            };
-            auto issue_dQ = [&]() {
+                mma_commit(BAR(C::DK_FULL));
+                // dQ += dS K_free, accumulated over every visit
+                const uint32_t kf = sb + C::kRing + slot_of(n, kJFree) * C::kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
                     mma_bf16_ss(tmem + C::kColDQ,
                                 sw128_desc(sb + C::kDS + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
-                                sw128_desc(kfree + k * 2048, C::kBox, 1024), idQ, k > 0);
+                                sw128_desc(kf + k * 2048, C::kBox, 1024), idQ, (n > 0 || k > 0));
                 }
-            };
-            bool ok = mbar_wait(BAR(C::K_FULL), 0, abort_flag);
-            if (ok && C::kQS >= 2) {
-                ok = mbar_wait(BAR(C::Q_FULL + 0), 0, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    issue_S(0);
-                }
-            }
-            for (int n = 0; n < N && ok; ++n) {
-                if (C::kQS >= 2) {
-                    if (n + 1 < N) {
-                        const int s1 = (n + 1) % C::kQS;
-                        if (!mbar_wait(BAR(C::Q_FULL + s1), ((n + 1) / C::kQS) & 1, abort_flag)) break;
-                        if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
-                        tc_fence_after();
-                        issue_S(n + 1);
-                    }
-                } else {
-                    if (!mbar_wait(BAR(C::Q_FULL + 0), n & 1, abort_flag)) break;
-                    if (n > 0 && !mbar_wait(BAR(C::S_FREE), (n - 1) & 1, abort_flag)) break;
-                    tc_fence_after();
-                    issue_S(n);
-                }
-                if (!mbar_wait(BAR(C::DS_FULL), n & 1, abort_flag)) break;
-                tc_fence_after();
-                issue_dK(n);
-                if (n > 0) {
-                    if (!mbar_wait(BAR(C::DQ_FREE), (n - 1) & 1, abort_flag)) break;
-                    tc_fence_after();
-                }
-                issue_dQ();
                 mma_commit(BAR(C::DS_FREE));
-                mma_commit(BAR(C::Q_EMPTY + n % C::kQS));
-                mma_commit(BAR(C::DQ_FULL));
+                mma_commit(BAR(C::K_EMPTY + slot_of(n, kJFree)));
             }
-            mma_commit(BAR(C::DK_FULL));
+            mma_commit(BAR(C::DQ_DONE));
             mma_commit(BAR(C::DONE));
             drain_wait(BAR(C::DONE), 0);
         }
     } else if (warp < kBwdComputeWarp0) {
-        // ================================================================ dQ flush warpgroup
-        const int quarter = warp;               // TMEM lanes 32*quarter.. = query rows
+        // ================================================================ dK flush warpgroup
+        const int quarter = warp;               // TMEM lanes 32*quarter.. = key rows
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         // this warp's two 4 KiB staging slots, each [4-column group (8)][lane (32)][4 floats]
         float4* slots = reinterpret_cast<float4*>(smem + C::kStage + warp * 2 * C::kStageSlot);
         const uint32_t slots_s = smem_u32(slots);
         int chunk = 0;                          // running chunk count: slot = chunk & 1
         for (int n = 0; n < N; ++n) {
-            int h, qt;
-            sched.visit(n, h, qt);
-            if (!mbar_wait(BAR(C::DQ_FULL), n & 1, abort_flag)) break;
+            const int kt = sched.key_tile(n);
+            if (!mbar_wait(BAR(C::DK_FULL), n & 1, abort_flag)) break;
             tc_fence_after();
-            float* blk = p.dq_ws + ((size_t)(b * p.Hq + h) * p.nqt + qt) * (128 * D) +
-                         (size_t)quarter * (32 * D);
+            float* blk = p.dk_ws + ((size_t)bhk * p.nkt + kt) * (128 * D) + (size_t)quarter * (32 * D);
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c, ++chunk) {
                 uint32_t v[32];
-                tmem_ld32(lane_base + C::kColDQ + c * 32, v);
+                tmem_ld32(lane_base + C::kColDK + c * 32, v);
                 tmem_wait_ld();
                 if (c == D / 32 - 1) {
                     tc_fence_before();
-                    mbar_arrive(BAR(C::DQ_FREE));   // the dQ columns are all in registers
+                    mbar_arrive(BAR(C::DK_FREE));   // the dK columns are all in registers
                 }
                 float4* slot = slots + (chunk & 1) * (C::kStageSlot / 16);
                 if (lane == 0) bulk_wait_read_le1();   // the slot's previous chunk was read
@@ -429,7 +427,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         // ================================================================ compute warpgroups
         const int wg = (warp - kBwdComputeWarp0) >> 2;   // key columns [32*wg, 32*wg + 32)
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;      // TMEM lane: query row (S) or key row (dK)
+        const int r = quarter * 32 + lane;      // TMEM lane = query row
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.sl2;
         const float scale = p.scale;
@@ -437,50 +435,37 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         uint8_t* ds_tile = smem + C::kDS;
         // this thread's 64 bytes of dS row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
         uint8_t* ds_row = ds_tile + (wg >> 1) * C::kBox + r * 128;
+        const int q = q0 + r;
+        // this row's statistics, for the CTA's whole life: a = LSE1*log2(e), bq = LSE2*log2(e)
+        // (mode 1) or LSE2 - LSE1 - KL (mode 2), g; rows past NQ get g = 0 (their dS is 0)
+        float a = 0.f, bq = 0.f, g = 0.f;
+        if (q < p.NQ) {
+            const size_t o = (size_t)bh * p.NQ + q;
+            const float L1 = p.lse1[o], L2 = p.lse2[o];
+            a = L1 * LOG2E;
+            bq = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
+            g = p.dkl[o];
+        }
+        // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf makes
+        // a row with g = 0 give exactly 0)
+        const bool folded = !__any_sync(0xffffffffu, g < 0.f);
+        if (folded) {
+            const float lg = log2f(g);
+            a -= lg;
+            if (mode1) bq -= lg;
+        }
+        const int kc0 = wg * 32;
         bool ok = true;
-        // per-row statistics of visit n for this thread's query row: ra = LSE1*log2(e),
-        // rb = LSE2*log2(e) (mode 1) or LSE2 - LSE1 - KL (mode 2), rg = g; rows past NQ
-        // get g = 0 (their dS is 0)
-        auto load_row_consts = [&](int n, float& ra, float& rb, float& rg) {
-            int h, qt;
-            sched.visit(n, h, qt);
-            const int q = qt * 128 + r;
-            ra = 0.f;
-            rb = 0.f;
-            rg = 0.f;
-            if (q < p.NQ) {
-                const size_t o = (size_t)(b * p.Hq + h) * p.NQ + q;
-                const float L1 = p.lse1[o], L2 = p.lse2[o];
-                ra = L1 * LOG2E;
-                rb = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
-                rg = p.dkl[o];
-            }
-        };
-        float na = 0.f, nb = 0.f, ng = 0.f;
-        if (N > 0) load_row_consts(0, na, nb, ng);
         for (int n = 0; n < N; ++n) {
-            int h, qt;
-            sched.visit(n, h, qt);
-            // this visit's statistics were loaded one iteration ago; start the next ones
-            const float ca = na, cb = nb, cg = ng;
-            if (n + 1 < N) load_row_consts(n + 1, na, nb, ng);
-            // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf
-            // makes a row with g = 0 give exactly 0)
-            const bool folded = !__any_sync(0xffffffffu, cg < 0.f);
-            float a = ca, bq = cb;
-            if (folded) {
-                const float lg = log2f(cg);
-                a = ca - lg;
-                if (mode1) bq = cb - lg;
-            }
+            const int kt = sched.key_tile(n);
+            const int k0 = kt * 128;
             // masked columns: keys past the diagonal of a causal diagonal tile, and
             // zero-filled keys past NK; columns k < lim of this warpgroup are valid
-            const int kc0 = wg * 32;
-            const bool need_mask = (p.causal && qt == kt) || (k0 + 128 > p.NK);
+            const bool need_mask = (p.causal && kt == qt) || (k0 + 128 > p.NK);
             int lim = 32;
             if (need_mask) {
                 lim = min(lim, p.NK - k0 - kc0);
-                if (p.causal && qt == kt) lim = min(lim, r - kc0 + 1);
+                if (p.causal && kt == qt) lim = min(lim, r - kc0 + 1);
             }
             if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
                 ok = false;
@@ -493,7 +478,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 tmem_ld16(lane_base + C::kColS1 + kc0, xa);
                 tmem_ld16(lane_base + C::kColS2 + kc0, ya);
                 tmem_wait_ld();
-                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, cg, lim, packed);
+                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, g, lim, packed);
             }
             {
                 uint32_t xa[16], ya[16];
@@ -502,7 +487,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(BAR(C::S_FREE));      // all of this thread's S columns are read
-                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, cg, lim - 16, packed + 8);
+                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, g, lim - 16, packed + 8);
             }
             if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
                 ok = false;
@@ -518,18 +503,19 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             fence_async_smem();
             mbar_arrive(BAR(C::DS_FULL));
         }
-        if (ok && mbar_wait(BAR(C::DK_FULL), 0, abort_flag)) {
+        // dQ of this query tile, accumulated over every visit: scale, round, store
+        if (ok && mbar_wait(BAR(C::DQ_DONE), 0, abort_flag)) {
             tc_fence_after();
-            constexpr int kCols = D / 4;          // dK columns per warpgroup
+            constexpr int kCols = D / 4;          // dQ columns per warpgroup
             uint32_t v[kCols];
             if constexpr (D == 128) {
-                tmem_ld32(lane_base + C::kColDK + wg * kCols, v);
+                tmem_ld32(lane_base + C::kColDQ + wg * kCols, v);
             } else {
-                tmem_ld16(lane_base + C::kColDK + wg * kCols, v);
+                tmem_ld16(lane_base + C::kColDQ + wg * kCols, v);
             }
             tmem_wait_ld();
-            if (k0 + r < p.NK) {
-                uint4* dst = reinterpret_cast<uint4*>(p.dk + ((size_t)bhk * p.NK + k0 + r) * D + wg * kCols);
+            if (q < p.NQ) {
+                uint4* dst = reinterpret_cast<uint4*>(p.dq + ((size_t)bh * p.NQ + q) * D + wg * kCols);
 #pragma unroll
                 for (int k = 0; k < kCols / 8; ++k) {
                     float f[8];
@@ -551,29 +537,30 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #undef BAR
 }
 
-// dq = bf16(scale * ws), un-blocking the tile-blocked workspace.  One thread = one query
-// row's 32-column chunk: it reads 8 float4 (coalesced across the 32 lanes of the chunk) and
-// writes 64 contiguous bytes of its dQ row.
+// out = bf16(scale * ws), un-blocking a tile-blocked fp32 workspace of `rows` rows per
+// plane (planes = B*Hkv for dK) and ntiles 128-row tiles per plane.  One thread = one row's
+// 32-column chunk: it reads 8 float4 (coalesced across the 32 lanes of the chunk) and
+// writes 64 contiguous bytes of its row.
 template <int D>
 __global__ void __launch_bounds__(256)
-streamkl_dq_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dq, int BH, int NQ,
-                           int nqt, float scale) {
+streamkl_tile_convert_kernel(const float* __restrict__ ws, uint16_t* __restrict__ out, int planes,
+                             int rows, int ntiles, float scale) {
     constexpr int kChunks = D / 32;
-    const size_t total = (size_t)BH * nqt * 128 * kChunks;   // (bh, tile, quarter, chunk, lane)
+    const size_t total = (size_t)planes * ntiles * 128 * kChunks;   // (plane, tile, quarter, chunk, lane)
     for (size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x; t < total;
          t += (size_t)gridDim.x * blockDim.x) {
         const int lane = (int)(t & 31);
         const size_t u = t >> 5;
         const int c = (int)(u % kChunks);
         const int quarter = (int)((u / kChunks) & 3);
-        const size_t blk = u / kChunks / 4;        // bh * nqt + qt
-        const int qt = (int)(blk % nqt);
-        const size_t bh = blk / nqt;
-        const int q = qt * 128 + quarter * 32 + lane;
-        if (q >= NQ) continue;
+        const size_t blk = u / kChunks / 4;        // plane * ntiles + tile
+        const int tile = (int)(blk % ntiles);
+        const size_t plane = blk / ntiles;
+        const int row = tile * 128 + quarter * 32 + lane;
+        if (row >= rows) continue;
         const float4* src = reinterpret_cast<const float4*>(
             ws + blk * (128 * D) + (size_t)(quarter * kChunks + c) * 1024) + lane;
-        uint4* dst = reinterpret_cast<uint4*>(dq + (bh * NQ + q) * D + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(out + (plane * rows + row) * D + c * 32);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float4 a = src[(2 * k) * 32];

@@ -98,25 +98,25 @@ int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
 }
 
 template <int D, bool SHARED>
-int launch_bwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
+int launch_bwd(int mode, const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                const CUtensorMap& k2, const skl::BwdParams& p, int grid, size_t ws_bytes,
-               uint16_t* dq, cudaStream_t st) {
-    auto kern = p.mode == 1 ? skl::streamkl_bwd_kernel<D, SHARED, 1> : skl::streamkl_bwd_kernel<D, SHARED, 2>;
+               uint16_t* dk, cudaStream_t st) {
+    auto kern = mode == 1 ? skl::streamkl_bwd_kernel<D, SHARED, 1> : skl::streamkl_bwd_kernel<D, SHARED, 2>;
     constexpr int smem = skl::BwdCfg<D, SHARED>::kSmem;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    cudaError_t e = cudaMemsetAsync(p.dq_ws, 0, ws_bytes, st);
+    cudaError_t e = cudaMemsetAsync(p.dk_ws, 0, ws_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "workspace memset");
     kern<<<grid, skl::kBwdThreads, smem, st>>>(q1, q2, k1, k2, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_bwd launch");
-    const size_t threads = (size_t)p.B * p.Hq * p.nqt * 128 * (D / 32);
+    const size_t threads = (size_t)p.B * p.Hkv * p.nkt * 128 * (D / 32);
     size_t blocks = (threads + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    skl::streamkl_dq_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(p.dq_ws, dq, p.B * p.Hq,
-                                                                        p.NQ, p.nqt, p.scale);
+    skl::streamkl_tile_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(p.dk_ws, dk, p.B * p.Hkv,
+                                                                          p.NK, p.nkt, p.scale);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dq convert launch");
+    if (e != cudaSuccess) return cuda_fail(e, "dk convert launch");
     return STREAMKL_OK;
 }
 
@@ -185,10 +185,10 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
                   : launch_fwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
 }
 
-size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d) {
-    if (B < 1 || Hq < 1 || NQ < 1 || (d != 64 && d != 128)) return 0;
-    const size_t rows = (size_t)(NQ + 127) / 128 * 128;   // whole 128-row query tiles
-    return (size_t)B * Hq * rows * d * sizeof(float);
+size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || NQ < 1 || NK < 1 || (d != 64 && d != 128)) return 0;
+    const size_t rows = (size_t)(NK + 127) / 128 * 128;   // whole 128-row key tiles
+    return (size_t)B * Hkv * rows * d * sizeof(float);
 }
 
 int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
@@ -201,7 +201,7 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
         return STREAMKL_ERR_INVALID_ARG;
     int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
     if (rc) return rc;
-    if (workspace_bytes < streamkl_bwd_workspace_bytes(B, Hq, NQ, d)) return STREAMKL_ERR_INVALID_ARG;
+    if (workspace_bytes < streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d)) return STREAMKL_ERR_INVALID_ARG;
     const void* ptrs[] = {q1, k1, q2, k2, kl, lse1, lse2, dkl, dq, dk, workspace};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return STREAMKL_ERR_UNSUPPORTED;
@@ -214,24 +214,23 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
     skl::BwdParams p;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NQ = NQ; p.NK = NK;
     p.causal = causal ? 1 : 0;
-    p.mode = mode;
     p.nkt = (NK + 127) / 128;
     p.nqt = (NQ + 127) / 128;
     p.sl2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.kl = kl; p.lse1 = lse1; p.lse2 = lse2; p.dkl = dkl;
-    p.dq_ws = static_cast<float*>(workspace);
-    p.dk = dk;
-    const long long grid = (long long)B * Hkv * p.nkt;
+    p.dk_ws = static_cast<float*>(workspace);
+    p.dq = dq;
+    const long long grid = (long long)B * Hq * p.nqt;
     if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
-    const size_t ws = streamkl_bwd_workspace_bytes(B, Hq, NQ, d);
+    const size_t ws = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128) {
-        return shared ? launch_bwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st)
-                      : launch_bwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st);
+        return shared ? launch_bwd<128, true>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
+                      : launch_bwd<128, false>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
     }
-    return shared ? launch_bwd<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st)
-                  : launch_bwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, ws, dq, st);
+    return shared ? launch_bwd<64, true>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
+                  : launch_bwd<64, false>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
 }
 
 }  // extern "C"
@@ -286,7 +285,7 @@ extern "C" int streamkl_bwd_noalloc(int mode, const uint16_t* q1, const uint16_t
     if (mode != 1 && mode != 2) return STREAMKL_ERR_INVALID_ARG;
     int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
     if (rc) return rc;
-    const size_t need = streamkl_bwd_workspace_bytes(B, Hq, NQ, d);
+    const size_t need = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d);
     if (need == 0 || need > STREAMKL_NOALLOC_SCRATCH_BYTES) {
         snprintf(t_last_cuda_error, sizeof(t_last_cuda_error),
                  "streamkl_bwd_noalloc: needs %zu bytes of scratch, the built-in buffer holds %zu",

@@ -263,7 +263,7 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
     kl, l1, l2 = (torch.empty((B, Hq, NQ), device=dev) for _ in range(3))
     g = {m: (torch.empty_like(t["q1"]), torch.empty_like(t["k1"])) for m in (1, 2)}
-    ws = torch.empty(binding.streamkl_bwd_workspace_bytes(B, Hq, NQ, d) // 4, device=dev)
+    ws = torch.empty(binding.streamkl_bwd_workspace_bytes(B, Hq, w.Hkv, NQ, w.NK, d) // 4, device=dev)
 
     def fwd():
         binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal,
@@ -398,7 +398,7 @@ def run_gpu(args):
                      "note": "achieved = algorithmic FLOPs per call / CUDA-event duration of the "
                              "call on its stream%s" % (
                                  "; the backward call also runs the dQ-workspace memset and the "
-                                 "dQ convert kernel" if dom.startswith("bwd") else "")},
+                                 "dK convert kernel" if dom.startswith("bwd") else "")},
         "clocks": clk,
         "gpu_launches": 5 * args.steps,
         "e2e": e2e,

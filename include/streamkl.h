@@ -68,10 +68,11 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
                  float* kl, float* lse1, float* lse2, void* stream);
 
 /*
- * Bytes of fp32 workspace streamkl_bwd needs: B*Hq*ceil(NQ/128)*128*d*4 (the dQ
- * accumulator, whole 128-row query tiles).  Returns 0 for sizes outside the supported range.
+ * Bytes of fp32 workspace streamkl_bwd needs for these sizes: B*Hkv*ceil(NK/128)*128*d*4
+ * (the dK accumulator, whole 128-row key tiles).  Returns 0 for sizes outside the supported
+ * range.
  */
-size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d);
+size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d);
 
 /*
  * Backward of sum_i dkl[i] * KL_i, recomputing P_t = exp(S_t - LSE_t) tile by tile from the
@@ -90,7 +91,7 @@ size_t streamkl_bwd_workspace_bytes(int B, int Hq, int NQ, int d);
  *   dq             : bf16 [B,Hq,NQ,d] output, overwritten.
  *   dk             : bf16 [B,Hkv,NK,d] output, overwritten.
  *   workspace      : caller-owned device buffer of at least
- *                    streamkl_bwd_workspace_bytes(B,Hq,NQ,d) bytes, 16-byte aligned; its
+ *                    streamkl_bwd_workspace_bytes(B,Hq,Hkv,NQ,NK,d) bytes, 16-byte aligned; its
  *                    contents on entry do not matter and are undefined on exit.  Two calls
  *                    that run at the same time need two workspaces.
  */
@@ -114,7 +115,7 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
  * device-wide synchronisation that cudaMalloc/cudaFree can cause.
  *
  * Same arguments, semantics and outputs as streamkl_bwd, minus workspace/workspace_bytes:
- * the fp32 dQ accumulator lives in a fixed STREAMKL_NOALLOC_SCRATCH_BYTES (32 MiB) buffer
+ * the fp32 dK accumulator lives in a fixed STREAMKL_NOALLOC_SCRATCH_BYTES (32 MiB) buffer
  * compiled into the library as a static device array.  Every GPU on which the library is
  * loaded holds that buffer until the process exits.
  *  - Sizes whose workspace (streamkl_bwd_workspace_bytes) exceeds the buffer return

@@ -44,17 +44,21 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_bytes(lib):
-    assert binding.streamkl_bwd_workspace_bytes(1, 32, 16384, 128) == 32 * 16384 * 128 * 4
-    assert binding.streamkl_bwd_workspace_bytes(2, 3, 5, 64) == 2 * 3 * 128 * 64 * 4   # whole tiles
-    assert binding.streamkl_bwd_workspace_bytes(1, 1, 129, 128) == 256 * 128 * 4
-    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 96) == 0
-    assert binding.streamkl_bwd_workspace_bytes(0, 1, 1, 64) == 0
+    # the dK accumulator: B * Hkv * whole 128-row key tiles * d fp32
+    assert binding.streamkl_bwd_workspace_bytes(1, 32, 32, 16384, 16384, 128) == 32 * 16384 * 128 * 4
+    assert binding.streamkl_bwd_workspace_bytes(2, 6, 3, 5, 5, 64) == 2 * 3 * 128 * 64 * 4
+    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 7, 129, 128) == 256 * 128 * 4
+    assert binding.streamkl_bwd_workspace_bytes(4, 32, 8, 2048, 32768, 64) == 4 * 8 * 32768 * 64 * 4
+    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 1, 1, 96) == 0
+    assert binding.streamkl_bwd_workspace_bytes(0, 1, 1, 1, 1, 64) == 0
 
 
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced: every call below fails its checks first
+HOST_REJECTIONS = (binding.ERR_INVALID_ARG, binding.ERR_UNSUPPORTED)
 
 
 def fwd_call(**kw):
+    assert kw.pop("_expect") in HOST_REJECTIONS   # never reach a launch with fake pointers
     args = dict(q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, B=1, Hq=2, Hkv=1, NQ=8, NK=8, d=64,
                 scale=0.125, causal=0, kl=FAKE, lse1=FAKE, lse2=FAKE, stream=0)
     args.update(kw)
@@ -78,13 +82,17 @@ def fwd_call(**kw):
     (dict(B=1 << 20, Hq=1 << 6, Hkv=1, NQ=1 << 6), binding.ERR_UNSUPPORTED),
 ])
 def test_fwd_rejects_on_host(lib, kw, want):
-    assert fwd_call(**kw) == want
+    assert fwd_call(_expect=want, **kw) == want
+
+
+WS_NEED = 1 * 1 * 128 * 64 * 4   # B=1, Hkv=1, one 128-row key tile, d=64
 
 
 def bwd_call(**kw):
+    assert kw.pop("_expect") in HOST_REJECTIONS   # never reach a launch with fake pointers
     args = dict(mode=1, q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, kl=FAKE, lse1=FAKE, lse2=FAKE,
                 dkl=FAKE, B=1, Hq=2, Hkv=1, NQ=8, NK=8, d=64, scale=0.125, causal=0, dq=FAKE,
-                dk=FAKE, workspace=FAKE, workspace_bytes=2 * 128 * 64 * 4, stream=0)
+                dk=FAKE, workspace=FAKE, workspace_bytes=WS_NEED, stream=0)
     args.update(kw)
     return binding.streamkl_bwd(**args)
 
@@ -94,14 +102,15 @@ def bwd_call(**kw):
     (dict(mode=3), binding.ERR_INVALID_ARG),
     (dict(dq=None), binding.ERR_INVALID_ARG),
     (dict(workspace=None), binding.ERR_INVALID_ARG),
-    (dict(workspace_bytes=2 * 128 * 64 * 4 - 4), binding.ERR_INVALID_ARG),
+    (dict(workspace_bytes=WS_NEED - 4), binding.ERR_INVALID_ARG),
     (dict(d=32), binding.ERR_UNSUPPORTED),
     (dict(causal=1, NK=7), binding.ERR_UNSUPPORTED),
     (dict(dk=FAKE + 2), binding.ERR_UNSUPPORTED),
     (dict(workspace=FAKE + 4), binding.ERR_UNSUPPORTED),
 ])
 def test_bwd_rejects_on_host(lib, kw, want):
-    assert bwd_call(**kw) == want
+    assert binding.streamkl_bwd_workspace_bytes(1, 2, 1, 8, 8, 64) == WS_NEED
+    assert bwd_call(_expect=want, **kw) == want
 
 
 def test_header_is_plain_c():

@@ -75,7 +75,7 @@ def test_shapes(case, mode):
 def test_workspace_contents_do_not_matter():
     w = inputs.custom(1, 2, 2, 384, 384, 128, True, True, seed=4)
     t = inputs.make(w, device="cuda")
-    n = binding.streamkl_bwd_workspace_bytes(1, 2, 384, 128) // 4
+    n = binding.streamkl_bwd_workspace_bytes(1, 2, 2, 384, 384, 128) // 4
     ws = torch.full((n,), float("nan"), device="cuda")
     a = gpu_bwd(t, w, 1, workspace=ws)
     ws.fill_(1e30)
@@ -105,7 +105,7 @@ def test_extra_memory_is_only_the_workspace():
     w = inputs.custom(1, 8, 8, 2048, 2048, 128, True, True, seed=9)
     t = inputs.make(w, device="cuda")
     kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], causal=True)
-    n = binding.streamkl_bwd_workspace_bytes(1, 8, 2048, 128) // 4
+    n = binding.streamkl_bwd_workspace_bytes(1, 8, 8, 2048, 2048, 128) // 4
     ws = torch.empty(n, device="cuda")
     out = (torch.empty_like(t["q1"]), torch.empty_like(t["k1"]))
     binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], causal=True, out=out, workspace=ws)

@@ -1,6 +1,6 @@
 """streamkl_bwd_noalloc: the backward for callers that may not allocate device memory (a
 framework allocator that owns the GPU, a fixed memory budget, no room for cudaMalloc's
-synchronisation).  It keeps the dQ accumulator in the library's built-in 32 MiB buffer
+synchronisation).  It keeps the dK accumulator in the library's built-in 32 MiB buffer
 instead of a caller workspace.  Checked here through the C ABI against streamkl_bwd with a
 torch-allocated workspace, on two calls in a row (the buffer keeps the previous call's
 contents, which must not leak into the next result)."""
@@ -21,7 +21,7 @@ def _fwd(t, w):
 
 def _with_workspace(mode, t, w, stats):
     dq, dk = torch.empty_like(t["q1"]), torch.empty_like(t["k1"])
-    ws = torch.empty(binding.streamkl_bwd_workspace_bytes(w.B, w.Hq, w.NQ, w.d) // 4, device="cuda")
+    ws = torch.empty(binding.streamkl_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.NQ, w.NK, w.d) // 4, device="cuda")
     rc = binding.streamkl_bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], *stats, t["dkl"], w.B, w.Hq,
                               w.Hkv, w.NQ, w.NK, w.d, w.scale, w.causal, dq, dk, ws,
                               ws.numel() * 4)
@@ -57,7 +57,7 @@ CASES = [
 def test_matches_workspace_backward_twice(case, mode):
     B, Hq, Hkv, NQ, NK, d, causal, shared = case
     w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=31 + NQ + d)
-    assert binding.streamkl_bwd_workspace_bytes(B, Hq, NQ, d) <= binding.NOALLOC_SCRATCH_BYTES
+    assert binding.streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d) <= binding.NOALLOC_SCRATCH_BYTES
     t = inputs.make(w, device="cuda")
     t["dkl"] = torch.rand(t["dkl"].shape, generator=torch.Generator().manual_seed(3)).cuda() + 0.5
     stats = _fwd(t, w)
@@ -71,9 +71,9 @@ def test_matches_workspace_backward_twice(case, mode):
 
 
 def test_rejects_problems_larger_than_the_buffer():
-    # 33 MiB of dQ accumulator: refused on the host before any launch
+    # 33 MiB of dK accumulator: refused on the host before any launch
     B, Hq, NQ, d = 1, 33, 2048, 128
-    assert binding.streamkl_bwd_workspace_bytes(B, Hq, NQ, d) > binding.NOALLOC_SCRATCH_BYTES
+    assert binding.streamkl_bwd_workspace_bytes(B, Hq, Hq, NQ, NQ, d) > binding.NOALLOC_SCRATCH_BYTES
     fake = 1 << 20
     rc = binding.streamkl_bwd_noalloc(1, fake, fake, fake, fake, fake, fake, fake, fake, B, Hq, Hq,
                                       NQ, NQ, d, 0.088, 1, fake, fake, stream=0)
