@@ -29,6 +29,7 @@ EXPORTS = (
     "streamkl_bwd_noalloc",
     "streamkl_status_string",
     "streamkl_device_status",
+    "streamkl_selftest_watchdog",
     "streamkl_last_cuda_error",
     "streamkl_version",
 )
@@ -70,6 +71,8 @@ def load(path=None):
     lib.streamkl_status_string.restype = ctypes.c_char_p
     lib.streamkl_device_status.argtypes = [vp]
     lib.streamkl_device_status.restype = i
+    lib.streamkl_selftest_watchdog.argtypes = [i, ctypes.POINTER(ctypes.c_longlong), vp]
+    lib.streamkl_selftest_watchdog.restype = i
     lib.streamkl_last_cuda_error.argtypes = []
     lib.streamkl_last_cuda_error.restype = ctypes.c_char_p
     lib.streamkl_version.argtypes = []
@@ -133,6 +136,13 @@ def streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d):
 
 def streamkl_device_status(stream=None):
     return load().streamkl_device_status(_stream(stream))
+
+
+def streamkl_selftest_watchdog(starve, stream=None):
+    """Runs the bounded-wait self-test; returns (status, [ns of wait 0, ns of wait 1])."""
+    ns = (ctypes.c_longlong * 2)()
+    rc = load().streamkl_selftest_watchdog(int(starve), ns, _stream(stream))
+    return rc, [ns[0], ns[1]]
 
 
 def status_string(status):

@@ -15,16 +15,19 @@
 //   tensor core : S1 = Q1 K1^T, S2 = Q2 K2^T               (TMEM, lane = query row)
 //   4 compute warpgroups: dS for 32 key columns each (thread = query row: the row's LSEs,
 //                 KL and g sit in registers for the CTA's whole life) -> bf16, written
-//                 once into a swizzled shared tile [query][key] that feeds both MMAs below
+//                 once into one of two swizzled shared tiles [query][key] (visit parity)
+//                 that feed both MMAs below
 //   tensor core : dQ += dS K_free    (dS read K-major; TMEM accumulator over all visits:
 //                                     dQ never leaves the chip until the end)
 //                 dKp  = dS^T Q_free (dS read MN-major; TMEM, lane = key)
-//   flush warpgroup: dKp from TMEM through a double-buffered shared staging area into an
-//                 fp32 dK workspace with bulk L2 reductions (cp.reduce.async.bulk .add.f32)
+//   flush warpgroup: dKp from TMEM into registers, then into an fp32 dK workspace with
+//                 16-byte vector reductions in L2 (red.global.add.v4.f32)
 // Streaming the key tile (32 KiB with shared keys) instead of the query pair keeps the
-// per-visit load small enough for a ring that prefetches two visits ahead, and the MMA
-// issuer looks one visit ahead: S of visit n+1 runs while the warpgroups turn S of visit n
-// into dS.
+// per-visit load small enough for a ring that prefetches two visits ahead; the MMA issuer
+// looks one visit ahead (S of visit n+1 runs while the warpgroups turn S of visit n into
+// dS), and the two dS tiles let the warpgroups write dS of visit n+1 while the dQ and dK
+// MMAs of visit n still read theirs, so the tensor core is handed work without waiting for
+// the write.
 //
 // The workspace is private to the library and tile-blocked: one contiguous 128 x d block
 // per (batch, KV head, key tile), laid out [lane quarter][32-column chunk][4-column group]
@@ -72,21 +75,21 @@ struct BwdCfg {
     static constexpr int kQ1 = 0;
     static constexpr int kQ2 = kTile;
     static constexpr int kRing = 2 * kTile;                        // slot s at kRing + s*kTile
-    static constexpr int kDS = kRing + kSlots * kTile;             // dS tile, 128 x 128 bf16
-    static constexpr int kStage = kDS + 128 * 128 * 2;             // dK staging: 4 warps x 2 x 4 KiB
-    static constexpr int kStageSlot = 4096;                        // 32 rows x 32 fp32 columns
-    static constexpr int kBar = kStage + 4 * 2 * kStageSlot;
+    static constexpr int kDS = kRing + kSlots * kTile;             // dS tiles, 2 x 128 x 128 bf16
+    static constexpr int kDSBuf = 128 * 128 * 2;                   // dS tile b at kDS + b*kDSBuf
+    static constexpr int kBar = kDS + 2 * kDSBuf;
     static constexpr int Q_FULL = 0;
     static constexpr int K_FULL = 1;                // + s
     static constexpr int K_EMPTY = 1 + kSlots;      // + s
     static constexpr int S_FULL = 1 + 2 * kSlots;
     static constexpr int S_FREE = S_FULL + 1;
-    static constexpr int DS_FULL = S_FULL + 2;
-    static constexpr int DS_FREE = S_FULL + 3;
-    static constexpr int DK_FULL = S_FULL + 4;
-    static constexpr int DK_FREE = S_FULL + 5;
-    static constexpr int DQ_DONE = S_FULL + 6;
-    static constexpr int DONE = S_FULL + 7;
+    // DS_FULL + b: dS tile b written by the compute warps AND the dK columns of the
+    // previous visit read out by the flush warps -- the one wait before dQ and dK
+    static constexpr int DS_FULL = S_FULL + 2;      // + b
+    static constexpr int DS_FREE = S_FULL + 4;      // + b
+    static constexpr int DK_FULL = S_FULL + 6;
+    static constexpr int DQ_DONE = S_FULL + 7;
+    static constexpr int DONE = S_FULL + 8;
     static constexpr int kNumBars = DONE + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kSmem = kMisc + 16 + 1024;
@@ -112,22 +115,11 @@ struct BwdSchedule {
     }
 };
 
-// dst[0..bytes) += src[0..bytes) in L2 (fp32 add), read from shared memory by the bulk copy
-// engine; completion tracked by this thread's bulk async-group.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
-                 ::"l"(dst), "r"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// At most one of this thread's bulk groups is still reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_le1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-// All of this thread's bulk groups have completed (global writes done).
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+// p[0..3] += (a, b, c, d) in L2, one 16-byte fp32 vector reduction (p 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(a)),
+                 "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -147,15 +139,41 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
-// dS of one query row over 16 key columns, packed to bf16 pairs.  x = S1 raw, y = S2 raw;
+// 8 consecutive fp32 TMEM columns of the thread's lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// tcgen05.wait::ld that also names the 16 registers the outstanding loads write, so that
+// no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[8], uint32_t (&b)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]),
+                   "+r"(a[6]), "+r"(a[7]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]),
+                   "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])
+                 :: "memory");
+}
+
+// Which of a chunk's four column pairs take their P2 exponential on the FMA pipe instead of
+// the exponential unit (mode 1 only; mode 2 has one exponential per element and leaves the
+// unit half idle).  Two of the chunk's eight exponential pairs = a quarter of the mode-1
+// exponentials.
+#ifndef SKL_BWD_EMU2
+#define SKL_BWD_EMU2 0x5
+#endif
+
+// dS of one query row over 8 key columns, packed to 4 bf16 pairs.  x = S1 raw, y = S2 raw;
 // a = LSE1*log2(e); b = LSE2*log2(e) (mode 1) or LSE2-LSE1-KL (mode 2); g = upstream
 // gradient.  FOLDED: g >= 0 has been folded into the exponents (a and, in mode 1, b
 // lowered by log2 g, so 2^(u - a) is already g*P) and g is not multiplied again.  Adjacent
 // columns are processed as fp32x2 pairs.  With MASKED, columns k >= lim are zero.
 template <int MODE, bool MASKED, bool FOLDED>
-__device__ __forceinline__ void ds_half(const uint32_t (&xa)[16], const uint32_t (&ya)[16],
-                                        float sl2, float scale, float a, float b, float g,
-                                        int lim, uint32_t* packed) {
+__device__ __forceinline__ void ds_chunk(const uint32_t (&xa)[8], const uint32_t (&ya)[8],
+                                         float sl2, float scale, float a, float b, float g,
+                                         int lim, uint32_t* packed) {
     const float2 sl = make_float2(sl2, sl2);
     const float2 na = make_float2(-a, -a);
     const float2 nb = make_float2(-b, -b);
@@ -164,7 +182,7 @@ __device__ __forceinline__ void ds_half(const uint32_t (&xa)[16], const uint32_t
     const float2 sc = make_float2(scale, scale);
     const float2 neg1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int pr = 0; pr < 8; ++pr) {
+    for (int pr = 0; pr < 4; ++pr) {
         const float2 xk = make_float2(__uint_as_float(xa[2 * pr]), __uint_as_float(xa[2 * pr + 1]));
         const float2 yk = make_float2(__uint_as_float(ya[2 * pr]), __uint_as_float(ya[2 * pr + 1]));
         const float2 u1 = __ffma2_rn(xk, sl, na);
@@ -172,7 +190,8 @@ __device__ __forceinline__ void ds_half(const uint32_t (&xa)[16], const uint32_t
         float2 v;
         if (MODE == 1) {
             const float2 u2 = __ffma2_rn(yk, sl, nb);
-            const float2 p2 = make_float2(ex2(u2.x), ex2(u2.y));
+            const float2 p2 = ((SKL_BWD_EMU2 >> pr) & 1) ? ex2_poly2(u2)
+                                                         : make_float2(ex2(u2.x), ex2(u2.y));
             v = __ffma2_rn(p1, neg1, p2);                  // (g)P2 - (g)P1
             if (!FOLDED) v = __fmul2_rn(v, gg);
         } else {
@@ -189,15 +208,15 @@ __device__ __forceinline__ void ds_half(const uint32_t (&xa)[16], const uint32_t
 }
 
 template <int MODE>
-__device__ __forceinline__ void ds_half_any(bool masked, bool folded, const uint32_t (&xa)[16],
-                                            const uint32_t (&ya)[16], float sl2, float scale,
-                                            float a, float b, float g, int lim, uint32_t* packed) {
+__device__ __forceinline__ void ds_chunk_any(bool masked, bool folded, const uint32_t (&xa)[8],
+                                             const uint32_t (&ya)[8], float sl2, float scale,
+                                             float a, float b, float g, int lim, uint32_t* packed) {
     if (folded) {
-        if (masked) ds_half<MODE, true, true>(xa, ya, sl2, scale, a, b, g, lim, packed);
-        else ds_half<MODE, false, true>(xa, ya, sl2, scale, a, b, g, 16, packed);
+        if (masked) ds_chunk<MODE, true, true>(xa, ya, sl2, scale, a, b, g, lim, packed);
+        else ds_chunk<MODE, false, true>(xa, ya, sl2, scale, a, b, g, 8, packed);
     } else {
-        if (masked) ds_half<MODE, true, false>(xa, ya, sl2, scale, a, b, g, lim, packed);
-        else ds_half<MODE, false, false>(xa, ya, sl2, scale, a, b, g, 16, packed);
+        if (masked) ds_chunk<MODE, true, false>(xa, ya, sl2, scale, a, b, g, lim, packed);
+        else ds_chunk<MODE, false, false>(xa, ya, sl2, scale, a, b, g, 8, packed);
     }
 }
 
@@ -250,10 +269,11 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         }
         mbar_init(BAR(C::S_FULL), 1);
         mbar_init(BAR(C::S_FREE), 32 * 4 * kBwdWG);
-        mbar_init(BAR(C::DS_FULL), 32 * 4 * kBwdWG);
-        mbar_init(BAR(C::DS_FREE), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(C::DS_FULL + b), 32 * 4 * kBwdWG + 128);
+            mbar_init(BAR(C::DS_FREE + b), 1);
+        }
         mbar_init(BAR(C::DK_FULL), 1);
-        mbar_init(BAR(C::DK_FREE), 128);
         mbar_init(BAR(C::DQ_DONE), 1);
         mbar_init(BAR(C::DONE), 1);
         *abort_flag = 0;
@@ -354,29 +374,26 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     tc_fence_after();
                     if (!issue_S(n + 1)) break;
                 }
-                if (!mbar_wait(BAR(C::DS_FULL), n & 1, abort_flag)) break;
+                const uint32_t ds = sb + C::kDS + (n & 1) * C::kDSBuf;
+                if (!mbar_wait(BAR(C::DS_FULL + (n & 1)), (n >> 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                if (n > 0) {
-                    if (!mbar_wait(BAR(C::DK_FREE), (n - 1) & 1, abort_flag)) break;
-                    tc_fence_after();
-                }
-                // dK partial of this key tile: dS^T Q_free (fresh every visit)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDK, sw128_desc(sb + C::kDS + k * 2048, C::kBox, 1024),
-                                sw128_desc(qfree + k * 2048, C::kBox, 1024), idK, k > 0);
-                }
-                mma_commit(BAR(C::DK_FULL));
-                // dQ += dS K_free, accumulated over every visit
+                // dQ += dS K_free, accumulated over every visit; it does not wait for the flush
                 const uint32_t kf = sb + C::kRing + slot_of(n, kJFree) * C::kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
                     mma_bf16_ss(tmem + C::kColDQ,
-                                sw128_desc(sb + C::kDS + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
+                                sw128_desc(ds + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
                                 sw128_desc(kf + k * 2048, C::kBox, 1024), idQ, (n > 0 || k > 0));
                 }
-                mma_commit(BAR(C::DS_FREE));
                 mma_commit(BAR(C::K_EMPTY + slot_of(n, kJFree)));
+                // dK partial of this key tile: dS^T Q_free (fresh every visit)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
+                    mma_bf16_ss(tmem + C::kColDK, sw128_desc(ds + k * 2048, C::kBox, 1024),
+                                sw128_desc(qfree + k * 2048, C::kBox, 1024), idK, k > 0);
+                }
+                mma_commit(BAR(C::DK_FULL));
+                mma_commit(BAR(C::DS_FREE + (n & 1)));
             }
             mma_commit(BAR(C::DQ_DONE));
             mma_commit(BAR(C::DONE));
@@ -386,43 +403,32 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         // ================================================================ dK flush warpgroup
         const int quarter = warp;               // TMEM lanes 32*quarter.. = key rows
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        // this warp's two 4 KiB staging slots, each [4-column group (8)][lane (32)][4 floats]
-        float4* slots = reinterpret_cast<float4*>(smem + C::kStage + warp * 2 * C::kStageSlot);
-        const uint32_t slots_s = smem_u32(slots);
-        int chunk = 0;                          // running chunk count: slot = chunk & 1
+        mbar_arrive(BAR(C::DS_FULL));               // visit 0 has no earlier dK to wait for
         for (int n = 0; n < N; ++n) {
             const int kt = sched.key_tile(n);
             if (!mbar_wait(BAR(C::DK_FULL), n & 1, abort_flag)) break;
             tc_fence_after();
-            float* blk = p.dk_ws + ((size_t)bhk * p.nkt + kt) * (128 * D) + (size_t)quarter * (32 * D);
+            // this lane's 16-byte groups of its key row: [chunk][group][lane][4] in the block
+            float* dst = p.dk_ws + ((size_t)bhk * p.nkt + kt) * (128 * D) + (size_t)quarter * (32 * D) +
+                         lane * 4;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c, ++chunk) {
-                uint32_t v[32];
-                tmem_ld32(lane_base + C::kColDK + c * 32, v);
+            for (int c = 0; c < D / 32; c += 2) {
+                uint32_t v[2][32];
+                tmem_ld32(lane_base + C::kColDK + c * 32, v[0]);
+                tmem_ld32(lane_base + C::kColDK + c * 32 + 32, v[1]);
                 tmem_wait_ld();
-                if (c == D / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(BAR(C::DK_FREE));   // the dK columns are all in registers
+                if (c + 2 == D / 32) {           // the dK columns are all in registers:
+                    tc_fence_before();           // visit n+1 may overwrite them
+                    mbar_arrive(BAR(C::DS_FULL + ((n + 1) & 1)));
                 }
-                float4* slot = slots + (chunk & 1) * (C::kStageSlot / 16);
-                if (lane == 0) bulk_wait_read_le1();   // the slot's previous chunk was read
-                __syncwarp();
 #pragma unroll
-                for (int g = 0; g < 8; ++g)
-                    slot[g * 32 + lane] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                                                      __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    bulk_reduce_add_f32(blk + c * (32 * 32), slots_s + (chunk & 1) * C::kStageSlot,
-                                        C::kStageSlot);
-                    bulk_commit();
-                }
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        red_add_v4(dst + (c + h) * (32 * 32) + g * 128, v[h][4 * g], v[h][4 * g + 1],
+                                   v[h][4 * g + 2], v[h][4 * g + 3]);
             }
         }
-        // every bulk reduction this warp started has landed before the CTA exits
-        if (lane == 0) bulk_wait_all();
-        __syncwarp();
     } else if (warp < kBwdComputeWarp0 + 4 * kBwdWG) {
         // ================================================================ compute warpgroups
         const int wg = (warp - kBwdComputeWarp0) >> 2;   // key columns [32*wg, 32*wg + 32)
@@ -432,9 +438,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         const float sl2 = p.sl2;
         const float scale = p.scale;
         const float LOG2E = 1.4426950408889634f;
-        uint8_t* ds_tile = smem + C::kDS;
-        // this thread's 64 bytes of dS row r: box (wg/2), 16-byte chunks 4*(wg&1)..+3
-        uint8_t* ds_row = ds_tile + (wg >> 1) * C::kBox + r * 128;
+        // this thread's 64 bytes of dS row r in tile 0: box (wg/2), 16-byte chunks 4*(wg&1)..+3
+        uint8_t* ds_row0 = smem + C::kDS + (wg >> 1) * C::kBox + r * 128;
         const int q = q0 + r;
         // this row's statistics, for the CTA's whole life: a = LSE1*log2(e), bq = LSE2*log2(e)
         // (mode 1) or LSE2 - LSE1 - KL (mode 2), g; rows past NQ get g = 0 (their dS is 0)
@@ -472,27 +477,33 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 break;
             }
             tc_fence_after();
+            // the warpgroup's 32 columns in four 8-column chunks: the load of chunk c+1 is in
+            // flight while chunk c is turned into dS, so only the first load's latency shows
             uint32_t packed[16];
-            {
-                uint32_t xa[16], ya[16];
-                tmem_ld16(lane_base + C::kColS1 + kc0, xa);
-                tmem_ld16(lane_base + C::kColS2 + kc0, ya);
-                tmem_wait_ld();
-                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, g, lim, packed);
+            uint32_t xa[2][8], ya[2][8];
+            tmem_ld8(lane_base + C::kColS1 + kc0, xa[0]);
+            tmem_ld8(lane_base + C::kColS2 + kc0, ya[0]);
+            tmem_wait_ld_regs(xa[0], ya[0]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c < 3) {
+                    tmem_ld8(lane_base + C::kColS1 + kc0 + 8 * (c + 1), xa[(c + 1) & 1]);
+                    tmem_ld8(lane_base + C::kColS2 + kc0 + 8 * (c + 1), ya[(c + 1) & 1]);
+                }
+                ds_chunk_any<MODE>(need_mask, folded, xa[c & 1], ya[c & 1], sl2, scale, a, bq, g,
+                                   lim - 8 * c, packed + 4 * c);
+                if (c < 3) tmem_wait_ld_regs(xa[(c + 1) & 1], ya[(c + 1) & 1]);
+                if (c == 2) {
+                    tc_fence_before();
+                    mbar_arrive(BAR(C::S_FREE));  // all of this thread's S columns are read
+                }
             }
-            {
-                uint32_t xa[16], ya[16];
-                tmem_ld16(lane_base + C::kColS1 + kc0 + 16, xa);
-                tmem_ld16(lane_base + C::kColS2 + kc0 + 16, ya);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(BAR(C::S_FREE));      // all of this thread's S columns are read
-                ds_half_any<MODE>(need_mask, folded, xa, ya, sl2, scale, a, bq, g, lim - 16, packed + 8);
-            }
-            if (n > 0 && !mbar_wait(BAR(C::DS_FREE), (n - 1) & 1, abort_flag)) {
+            // dS tile n&1 was last read by the MMAs of visit n-2
+            if (n > 1 && !mbar_wait(BAR(C::DS_FREE + (n & 1)), ((n >> 1) - 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
+            uint8_t* ds_row = ds_row0 + (n & 1) * C::kDSBuf;
             const int cbase = (wg & 1) * 4;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -501,7 +512,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
             }
             fence_async_smem();
-            mbar_arrive(BAR(C::DS_FULL));
+            mbar_arrive(BAR(C::DS_FULL + (n & 1)));
         }
         // dQ of this query tile, accumulated over every visit: scale, round, store
         if (ok && mbar_wait(BAR(C::DQ_DONE), 0, abort_flag)) {

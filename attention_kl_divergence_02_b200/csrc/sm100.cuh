@@ -57,12 +57,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase of parity `parity` of barrier `bar` to complete.  Gives up after
-// kWaitLimitNs, or as soon as this CTA's abort flag or the device status word is set;
-// a wait that runs out records STREAMKL_ERR_TIMEOUT (4) and raises the abort flag so the
-// other roles of the CTA stop too.  Returns false when it gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+// The spinning part of mbar_wait, kept out of line so that the common case (the phase is
+// already complete, or completes within the first probe) costs no call.
+__device__ __noinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     const unsigned long long t0 = globaltimer();
     while (true) {
 #pragma unroll 1
@@ -79,6 +76,18 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
             return false;
         }
     }
+}
+
+// Waits for the phase of parity `parity` of barrier `bar` to complete.  Gives up after
+// kWaitLimitNs, or as soon as this CTA's abort flag or the device status word is set;
+// a wait that runs out records STREAMKL_ERR_TIMEOUT (4) and raises the abort flag so the
+// other roles of the CTA stop too.  Returns false when it gave up.  The first probe is
+// inline: a thread that issues tensor-core work cannot afford a call per wait (the MMA
+// queue holds little more than one instruction, so every stall of the issuing thread
+// leaves the tensor pipe idle).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_spin(bar, parity, abort_flag);
 }
 
 // Wait used only while draining at exit (copies or MMAs this thread started must land

@@ -13,6 +13,7 @@
 #include "sm100.cuh"
 #include "fwd_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "watchdog.cuh"
 
 namespace {
 
@@ -150,6 +151,30 @@ int streamkl_device_status(void* stream) {
         if (e != cudaSuccess) return cuda_fail(e, "clear device status");
     }
     return v;
+}
+
+int streamkl_selftest_watchdog(int starve, long long* waited_ns, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned long long zero[3] = {0, 0, 0};
+    cudaError_t e = cudaMemcpyToSymbolAsync(skl::g_watchdog, zero, sizeof(zero), 0,
+                                            cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "watchdog reset");
+    skl::streamkl_watchdog_kernel<<<1, 64, 0, st>>>(starve);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "watchdog launch");
+    const int status = streamkl_device_status(stream);   // synchronises, reads, clears
+    if (status == STREAMKL_ERR_CUDA) return status;
+    unsigned long long res[3];
+    e = cudaMemcpyFromSymbol(res, skl::g_watchdog, sizeof(res));
+    if (e != cudaSuccess) return cuda_fail(e, "watchdog read");
+    if (waited_ns) {
+        waited_ns[0] = (long long)res[1];
+        waited_ns[1] = (long long)res[2];
+    }
+    // both waits must agree with the verdict: all passed (OK) or none did (TIMEOUT)
+    if (status == STREAMKL_OK && res[0] != 3ull) return STREAMKL_ERR_TIMEOUT;
+    if (status != STREAMKL_OK && res[0] != 0ull) return STREAMKL_ERR_CUDA;
+    return status;
 }
 
 int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,

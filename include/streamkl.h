@@ -144,6 +144,21 @@ const char* streamkl_status_string(int status);
  */
 int streamkl_device_status(void* stream);
 
+/*
+ * Self-test of the bounded waits that guard every pipeline kernel (no part of the KL
+ * computation).  Runs one small kernel on `stream` and waits for it: two threads wait on
+ * two mbarriers, the second starting 0.5 s after the first.
+ *   starve == 0: the barriers are completed before anyone waits; returns STREAMKL_OK.
+ *   starve != 0: nothing completes them.  The first wait gives up after the library's
+ *     wait limit (2 s), records STREAMKL_ERR_TIMEOUT and raises the CTA's abort flag; the
+ *     second wait sees the flag and gives up at once.  Returns STREAMKL_ERR_TIMEOUT.
+ * Nothing faults or traps; the context stays usable.  The device status word is read and
+ * cleared like streamkl_device_status does.  If waited_ns is not NULL it receives the
+ * nanoseconds each of the two waits took.  Returns STREAMKL_ERR_CUDA if a CUDA call
+ * failed.  Blocks the calling host thread for up to about 2.5 s.
+ */
+int streamkl_selftest_watchdog(int starve, long long* waited_ns, void* stream);
+
 /* Text of the last CUDA error the library saw on this host thread ("" if none). */
 const char* streamkl_last_cuda_error(void);
 

@@ -1,0 +1,52 @@
+"""Failure detection on the GPU without a fault: every pipeline wait of the library is
+bounded (a 2 s limit, then STREAMKL_ERR_TIMEOUT in the device status word and an abort
+flag that stops the CTA's other waits).  streamkl_selftest_watchdog runs that machinery on
+a barrier that nothing completes; the wait must run out, report the timeout to the host,
+stop the second waiter early, and leave the context usable for the real kernels."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_kl_divergence_02_b200 import binding, inputs
+
+from parity import KL_TOL, LSE_TOL
+
+pytestmark = pytest.mark.gpu
+
+LIMIT_NS = 2_000_000_000
+STAGGER_NS = 500_000_000
+
+
+def test_waits_pass_when_the_barrier_completes():
+    rc, ns = binding.streamkl_selftest_watchdog(0)
+    assert rc == binding.OK
+    assert max(ns) < 100_000_000
+    assert binding.streamkl_device_status() == binding.OK
+
+
+def test_starved_wait_times_out_and_stops_the_other_waiter():
+    rc, ns = binding.streamkl_selftest_watchdog(1)
+    assert rc == binding.ERR_TIMEOUT, binding.status_string(rc)
+    # the first wait ran out its own limit ...
+    assert LIMIT_NS <= ns[0] < LIMIT_NS + 500_000_000
+    # ... the second, started 0.5 s later, gave up when the first raised the abort flag,
+    # well before its own limit
+    assert ns[1] < LIMIT_NS - STAGGER_NS + 200_000_000
+    # the status word was read and cleared by the self-test
+    assert binding.streamkl_device_status() == binding.OK
+
+
+def test_context_usable_after_a_timeout():
+    rc, _ = binding.streamkl_selftest_watchdog(1)
+    assert rc == binding.ERR_TIMEOUT
+    w = inputs.WORKLOADS["tiny"]
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal)
+    assert binding.streamkl_device_status() == binding.OK
+    okl, ol1, ol2 = oracle.fwd(*[inputs.to_f64(t[k]) for k in ("q1", "k1", "q2", "k2")],
+                               scale=w.scale, causal=w.causal)
+    gkl = kl.double().cpu().numpy()
+    assert np.max(np.abs(gkl - okl) / np.maximum(1, np.abs(okl))) <= KL_TOL
+    assert np.max(np.abs(l1.double().cpu().numpy() - ol1)) <= LSE_TOL
+    assert np.max(np.abs(l2.double().cpu().numpy() - ol2)) <= LSE_TOL
