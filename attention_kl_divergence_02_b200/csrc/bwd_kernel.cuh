@@ -64,6 +64,7 @@ constexpr int kBwdWG = 4;          // compute warpgroups
 constexpr int kBwdComputeWarp0 = 4;
 constexpr int kBwdProducerWarp = 20;
 constexpr int kBwdMmaWarp = 21;
+constexpr int kBwdHeadGroup = 8;  // (batch, head) planes scheduled together
 
 template <int D, bool SHARED_K>
 struct BwdCfg {
@@ -238,10 +239,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: heaviest causal query tiles are handed out first
+    // ---- work unit.  The (batch, head) planes are taken kBwdHeadGroup at a time, and
+    // within a group the heaviest causal query tiles are handed out first.  The CTAs in
+    // flight then reduce into the dK blocks of a few KV heads only (a few MB per head), so
+    // the partial sums meet in L2 instead of going back and forth to DRAM.
     const int BH = p.B * p.Hq;
-    const int unit = blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    const int per_group = kBwdHeadGroup * p.nqt;
+    const int group = blockIdx.x / per_group;
+    const int gh = min(kBwdHeadGroup, BH - group * kBwdHeadGroup);   // planes in this group
+    const int r_in = blockIdx.x - group * per_group;
+    const int unit = r_in / gh;
+    const int bh = group * kBwdHeadGroup + r_in % gh;
     const int qt = p.causal ? (p.nqt - 1 - unit) : unit;
     const int b = bh / p.Hq;
     const int h = bh % p.Hq;
