@@ -64,7 +64,7 @@ constexpr int kBwdWG = 4;          // compute warpgroups
 constexpr int kBwdComputeWarp0 = 4;
 constexpr int kBwdProducerWarp = 20;
 constexpr int kBwdMmaWarp = 21;
-constexpr int kBwdHeadGroup = 8;  // (batch, head) planes scheduled together
+constexpr int kBwdHeadGroup = 2;   // (batch, head) planes scheduled together
 
 template <int D, bool SHARED_K>
 struct BwdCfg {
@@ -242,7 +242,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     // ---- work unit.  The (batch, head) planes are taken kBwdHeadGroup at a time, and
     // within a group the heaviest causal query tiles are handed out first.  The CTAs in
     // flight then reduce into the dK blocks of a few KV heads only (a few MB per head), so
-    // the partial sums meet in L2 instead of going back and forth to DRAM.
+    // the partial sums meet in L2 instead of going back and forth to DRAM (a group of 2
+    // measured best of 2, 4, 8 and 16 on the causal and GQA workloads).
     const int BH = p.B * p.Hq;
     const int per_group = kBwdHeadGroup * p.nqt;
     const int group = blockIdx.x / per_group;
@@ -348,12 +349,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             // S of visit n; returns false if a wait gave up
             auto issue_S = [&](int n) -> bool {
                 const uint32_t s1 = slot_of(n, kJ1);
+                const uint32_t s2 = SHARED_K ? s1 : slot_of(n, kJ2);
                 if (!mbar_wait(BAR(C::K_FULL + s1), fill_parity(n, kJ1), abort_flag)) return false;
-                uint32_t s2 = s1;
-                if (!SHARED_K) {
-                    s2 = slot_of(n, kJ2);
-                    if (!mbar_wait(BAR(C::K_FULL + s2), fill_parity(n, kJ2), abort_flag)) return false;
-                }
+                if (!SHARED_K && !mbar_wait(BAR(C::K_FULL + s2), fill_parity(n, kJ2), abort_flag))
+                    return false;
                 tc_fence_after();
                 const uint32_t k1s = sb + C::kRing + s1 * C::kTile;
                 const uint32_t k2s = sb + C::kRing + s2 * C::kTile;
