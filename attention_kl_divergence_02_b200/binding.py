@@ -24,6 +24,9 @@ ERR_TIMEOUT = 4
 
 EXPORTS = (
     "streamkl_fwd",
+    "streamkl_fwd_splitk",
+    "streamkl_fwd_splits",
+    "streamkl_fwd_splitk_workspace_bytes",
     "streamkl_bwd",
     "streamkl_bwd_workspace_bytes",
     "streamkl_bwd_noalloc",
@@ -59,6 +62,12 @@ def load(path=None):
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.streamkl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
     lib.streamkl_fwd.restype = i
+    lib.streamkl_fwd_splitk.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp, vp, vp, vp, sz, vp]
+    lib.streamkl_fwd_splitk.restype = i
+    lib.streamkl_fwd_splits.argtypes = [i, i, i, i]
+    lib.streamkl_fwd_splits.restype = i
+    lib.streamkl_fwd_splitk_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.streamkl_fwd_splitk_workspace_bytes.restype = sz
     lib.streamkl_bwd.argtypes = ([i, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
                                   vp, vp, vp, sz, vp])
     lib.streamkl_bwd.restype = i
@@ -104,6 +113,22 @@ def streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, kl, lse1,
     return load().streamkl_fwd(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), B, Hq, Hkv, NQ, NK, d,
                                float(scale), int(bool(causal)), _ptr(kl), _ptr(lse1), _ptr(lse2),
                                _stream(stream))
+
+
+def streamkl_fwd_splitk(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, kl, lse1, lse2,
+                        workspace, workspace_bytes, stream=None):
+    return load().streamkl_fwd_splitk(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), B, Hq, Hkv, NQ, NK, d,
+                                      float(scale), int(bool(causal)), int(splits), _ptr(kl),
+                                      _ptr(lse1), _ptr(lse2), _ptr(workspace), int(workspace_bytes),
+                                      _stream(stream))
+
+
+def streamkl_fwd_splits(B, Hq, NQ, NK):
+    return load().streamkl_fwd_splits(B, Hq, NQ, NK)
+
+
+def streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits):
+    return load().streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits)
 
 
 def streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale, causal,
@@ -184,6 +209,27 @@ def fwd(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
     rc = streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, *out, stream=stream)
     if rc != OK:
         raise StreamKLError(rc, "streamkl_fwd")
+    return out
+
+
+def fwd_splitk(q1, k1, q2, k2, scale=None, causal=False, splits=0, out=None, workspace=None,
+               stream=None):
+    """Split-K forward (key ranges merged exactly); same outputs as fwd.  splits = 0 lets
+    the library choose; `workspace` (fp32 tensor) is allocated here when not given."""
+    import torch
+    _check_inputs(q1, k1, q2, k2)
+    B, Hq, Hkv, NQ, NK, d = _dims(q1, k1)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = tuple(torch.empty((B, Hq, NQ), dtype=torch.float32, device=q1.device) for _ in range(3))
+    need = streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q1.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = streamkl_fwd_splitk(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, *out,
+                             workspace, wbytes, stream=stream)
+    if rc != OK:
+        raise StreamKLError(rc, "streamkl_fwd_splitk")
     return out
 
 

@@ -18,6 +18,13 @@
 // 32 rows that live in its lane quarter.
 //
 // Scores are kept in base-2 units: u = s_raw * scale * log2(e), where s_raw = <q, k>.
+//
+// Split-K (for few query rows and many keys, where one CTA per query block leaves most SMs
+// idle; the technical summary's "3. Otimizações de Kernel de GPU" names it for small N_Q):
+// with splits > 1 the key tiles are cut into ranges of kps tiles, CTA (block, split) folds
+// only its range, and instead of finishing it stores the five scalars of each row; the
+// merge kernel below combines the ranges exactly (each rescaled to the common maximum, the
+// same correction the online recurrence applies tile by tile).
 #pragma once
 
 #include "sm100.cuh"
@@ -33,6 +40,9 @@ struct FwdParams {
     float* kl;
     float* lse1;
     float* lse2;
+    int splits;    // key ranges per query block (1 = no split)
+    int kps;       // key tiles per range
+    float* part;   // splits > 1: partial state [splits][5][B*Hq*NQ]: m1, l1, m2, l2, acc
 };
 
 constexpr int kFwdThreads = 384;
@@ -180,10 +190,13 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: heaviest causal query blocks are handed out first
+    // ---- work unit: heaviest causal query blocks are handed out first; the key ranges of a
+    // query block are neighbours in the grid
     const int BH = p.B * p.Hq;
-    const int unit = blockIdx.x / BH;
-    const int bh = blockIdx.x % BH;
+    const int sp = blockIdx.x % p.splits;
+    const int ub = blockIdx.x / p.splits;
+    const int unit = ub / BH;
+    const int bh = ub % BH;
     const int qb = p.causal ? (p.n_qblk - 1 - unit) : unit;
     const int b = bh / p.Hq;
     const int h = bh % p.Hq;
@@ -203,7 +216,13 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         }
     }
     const int ntiles = nkt[1] > 0 ? 2 : 1;
-    const int nj = max(nkt[0], nkt[1]);
+    // this CTA's key tiles: [j0, jend[t]) for query tile t (empty when the range starts past
+    // the tile's causal end)
+    const int j0 = sp * p.kps;
+    int jend[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) jend[t] = max(j0, min(nkt[t], j0 + p.kps));
+    const int nj = max(jend[0], jend[1]);
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -247,7 +266,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             }
             uint32_t it = 0;
             bool ok = true;
-            for (int j = 0; j < nj && ok; ++j) {
+            for (int j = j0; j < nj && ok; ++j) {
 #pragma unroll
                 for (int w = 0; w < (SHARED_K ? 1 : 2); ++w) {
                     const uint32_t s = it % C::kSlots;
@@ -281,7 +300,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             for (int t = 0; t < ntiles && ok; ++t) ok = mbar_wait(BAR(C::Q_FULL + t), 0, abort_flag);
             tc_fence_after();
             uint32_t it = 0;
-            for (int j = 0; j < nj && ok; ++j) {
+            for (int j = j0; j < nj && ok; ++j) {
                 const uint32_t s1 = it % C::kSlots;
                 if (!mbar_wait(BAR(C::K_FULL + s1), (it / C::kSlots) & 1, abort_flag)) break;
                 ++it;
@@ -293,9 +312,9 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 }
                 tc_fence_after();
                 for (int t = 0; t < ntiles; ++t) {
-                    if (j >= nkt[t]) continue;
-                    if (j > 0) {
-                        if (!mbar_wait(BAR(C::S_FREE + t), (j - 1) & 1, abort_flag)) {
+                    if (j >= jend[t]) continue;
+                    if (j > j0) {
+                        if (!mbar_wait(BAR(C::S_FREE + t), (j - j0 - 1) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -338,12 +357,19 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             const float sl2 = p.sl2;
             float m1 = -1e30f, l1 = 0.f, m2 = -1e30f, l2 = 0.f, acc = 0.f;
             bool ok = true;
-            for (int j = 0; j < nkt[t]; ++j) {
-                if (!mbar_wait(BAR(C::S_FULL + t), j & 1, abort_flag)) {
+            // a warp whose 32 rows all lie past NQ only keeps the barrier protocol
+            const bool any_row = q0[t] + quarter * 32 < p.NQ;
+            for (int j = j0; j < jend[t]; ++j) {
+                if (!mbar_wait(BAR(C::S_FULL + t), (j - j0) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                if (!any_row) {
+                    tc_fence_before();
+                    mbar_arrive(BAR(C::S_FREE + t));
+                    continue;
+                }
                 const int kb = j * 128;
                 const bool masked = (kb + 128 > p.NK) || (p.causal && kb + 127 > q0[t]);
 #pragma unroll 1
@@ -368,7 +394,15 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     }
                 }
             }
-            if (ok && i < p.NQ) {
+            if (ok && i < p.NQ && p.splits > 1) {
+                const size_t R = (size_t)p.B * p.Hq * p.NQ;
+                float* dst = p.part + (size_t)sp * 5 * R + (size_t)bh * p.NQ + i;
+                dst[0] = m1;
+                dst[R] = l1;
+                dst[2 * R] = m2;
+                dst[3 * R] = l2;
+                dst[4 * R] = acc;
+            } else if (ok && i < p.NQ) {
                 const float LN2 = 0.6931471805599453f;
                 const float lg1 = log2f(l1);
                 const float lg2 = log2f(l2);
@@ -388,6 +422,38 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         tmem_dealloc(tmem, 512);
     }
 #undef BAR
+}
+
+// Combines the key ranges of a split forward, one thread per query row: with M = max_s m_s,
+// l = sum_s l_s 2^(m_s - M) and acc likewise (acc is rescaled with m1, as in the recurrence);
+// then the same finish as the unsplit kernel.  Ranges with no valid key for a row hold
+// m = -1e30, l = acc = 0 and drop out (2^(m_s - M) = 0).
+__global__ void __launch_bounds__(256)
+streamkl_splitk_merge_kernel(const float* __restrict__ part, int splits, long long R, float scale,
+                             float* __restrict__ kl, float* __restrict__ lse1, float* __restrict__ lse2) {
+    for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < R;
+         o += (long long)gridDim.x * blockDim.x) {
+        float M1 = -1e30f, M2 = -1e30f;
+        for (int s = 0; s < splits; ++s) {
+            M1 = fmaxf(M1, part[(s * 5 + 0) * R + o]);
+            M2 = fmaxf(M2, part[(s * 5 + 2) * R + o]);
+        }
+        float L1 = 0.f, L2 = 0.f, A = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* q = part + s * 5 * R + o;
+            const float a1 = ex2(q[0] - M1);
+            const float a2 = ex2(q[2 * R] - M2);
+            L1 = fmaf(q[R], a1, L1);
+            A = fmaf(q[4 * R], a1, A);
+            L2 = fmaf(q[3 * R], a2, L2);
+        }
+        const float LN2 = 0.6931471805599453f;
+        const float lg1 = log2f(L1);
+        const float lg2 = log2f(L2);
+        lse1[o] = (M1 + lg1) * LN2;
+        lse2[o] = (M2 + lg2) * LN2;
+        kl[o] = scale * A / L1 + ((M2 - M1) + (lg2 - lg1)) * LN2;
+    }
 }
 
 }  // namespace skl

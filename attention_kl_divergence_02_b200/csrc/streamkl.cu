@@ -7,7 +7,9 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "streamkl.h"
 #include "sm100.cuh"
@@ -177,17 +179,26 @@ int streamkl_selftest_watchdog(int starve, long long* waited_ns, void* stream) {
     return status;
 }
 
-int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
-                 int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
-                 float* kl, float* lse1, float* lse2, void* stream) {
-    if (!q1 || !k1 || !q2 || !k2 || !kl || !lse1 || !lse2) return STREAMKL_ERR_INVALID_ARG;
-    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
-    if (rc) return rc;
-    if (!aligned16(q1) || !aligned16(k1) || !aligned16(q2) || !aligned16(k2) || !aligned16(kl) ||
-        !aligned16(lse1) || !aligned16(lse2))
-        return STREAMKL_ERR_UNSUPPORTED;
+}  // extern "C"
+
+namespace {
+
+constexpr int kNumSMs = 148;
+
+// Key tiles per range for `splits` ranges, and the number of non-empty ranges that gives.
+void split_ranges(int NK, int splits, int* kps, int* used) {
+    const int nkt = (NK + 127) / 128;
+    const int s = std::max(1, std::min(splits, nkt));
+    *kps = (nkt + s - 1) / s;
+    *used = (nkt + *kps - 1) / *kps;
+}
+
+int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2, int B,
+             int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal, int splits, float* kl,
+             float* lse1, float* lse2, float* part, void* stream) {
     const bool shared = (k1 == k2);
     CUtensorMap mq1, mq2, mk1, mk2;
+    int rc;
     if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d))) return rc;
     if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d))) return rc;
     if ((rc = make_map(&mk1, k1, (long long)B * Hkv, NK, d))) return rc;
@@ -199,15 +210,97 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
     p.sl2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.kl = kl; p.lse1 = lse1; p.lse2 = lse2;
-    const long long grid = (long long)B * Hq * p.n_qblk;
+    split_ranges(NK, splits, &p.kps, &p.splits);
+    p.part = p.splits > 1 ? part : nullptr;
+    const long long grid = (long long)B * Hq * p.n_qblk * p.splits;
     if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128) {
-        return shared ? launch_fwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
-                      : launch_fwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+        rc = shared ? launch_fwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                    : launch_fwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+    } else {
+        rc = shared ? launch_fwd<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                    : launch_fwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
     }
-    return shared ? launch_fwd<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
-                  : launch_fwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+    if (rc || p.splits == 1) return rc;
+    const long long R = (long long)B * Hq * NQ;
+    const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * kNumSMs);
+    skl::streamkl_splitk_merge_kernel<<<mgrid, 256, 0, st>>>(part, p.splits, R, scale, kl, lse1, lse2);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+    return STREAMKL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
+                 int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                 float* kl, float* lse1, float* lse2, void* stream) {
+    if (!q1 || !k1 || !q2 || !k2 || !kl || !lse1 || !lse2) return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    if (!aligned16(q1) || !aligned16(k1) || !aligned16(q2) || !aligned16(k2) || !aligned16(kl) ||
+        !aligned16(lse1) || !aligned16(lse2))
+        return STREAMKL_ERR_UNSUPPORTED;
+    return fwd_impl(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, 1, kl, lse1, lse2,
+                    nullptr, stream);
+}
+
+int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
+    if (B < 1 || Hq < 1 || NQ < 1 || NK < 1) return 1;
+    const long long blocks = (long long)B * Hq * ((NQ + 255) / 256);
+    const int nkt = (NK + 127) / 128;
+    if (blocks >= kNumSMs || nkt < 2) return 1;
+    // time model: waves of one CTA per SM, each CTA ~ its key tiles + 2 tiles of fixed cost
+    // (query load, pipeline fill and drain); the fewest ranges within 3 % of the best
+    double best = 1e300;
+    int best_s = 1;
+    std::vector<double> cost(65, 0.0);
+    for (int s = 1; s <= std::min(nkt, 64); ++s) {
+        int kps, used;
+        split_ranges(NK, s, &kps, &used);
+        const long long ctas = blocks * used;
+        const double waves = (double)((ctas + kNumSMs - 1) / kNumSMs);
+        cost[s] = waves * (kps + 2);
+        if (cost[s] < best) best = cost[s];
+    }
+    for (int s = 1; s <= std::min(nkt, 64); ++s) {
+        if (cost[s] <= best * 1.03) {
+            best_s = s;
+            break;
+        }
+    }
+    int kps, used;
+    split_ranges(NK, best_s, &kps, &used);
+    return used;
+}
+
+size_t streamkl_fwd_splitk_workspace_bytes(int B, int Hq, int NQ, int NK, int splits) {
+    if (B < 1 || Hq < 1 || NQ < 1 || NK < 1 || splits < 0) return 0;
+    if (splits == 0) splits = streamkl_fwd_splits(B, Hq, NQ, NK);
+    int kps, used;
+    split_ranges(NK, splits, &kps, &used);
+    if (used <= 1) return 0;
+    return (size_t)used * 5 * B * Hq * NQ * sizeof(float);
+}
+
+int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
+                        const uint16_t* k2, int B, int Hq, int Hkv, int NQ, int NK, int d,
+                        float scale, int causal, int splits, float* kl, float* lse1, float* lse2,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q1 || !k1 || !q2 || !k2 || !kl || !lse1 || !lse2 || splits < 0) return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    if (!aligned16(q1) || !aligned16(k1) || !aligned16(q2) || !aligned16(k2) || !aligned16(kl) ||
+        !aligned16(lse1) || !aligned16(lse2) || !aligned16(workspace))
+        return STREAMKL_ERR_UNSUPPORTED;
+    if (splits == 0) splits = streamkl_fwd_splits(B, Hq, NQ, NK);
+    const size_t need = streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return STREAMKL_ERR_INVALID_ARG;
+    return fwd_impl(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, kl, lse1, lse2,
+                    static_cast<float*>(workspace), stream);
 }
 
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d) {

@@ -413,6 +413,92 @@ def run_gpu(args):
     return 0
 
 
+def run_decode(args):
+    """Split-K forward on the decode workload (one query row per head, 32768 keys): bound by
+    streaming the keys from HBM, so it reports GB/s of algorithmic traffic against the
+    measured copy bandwidth, and the unsplit forward beside it."""
+    import torch
+
+    from attention_kl_divergence_02_b200 import binding, inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--decode measures one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    binding.load()
+    w = inputs.WORKLOADS["decode"]
+    t = inputs.make(w, device=dev)
+    B, Hq, NQ, NK, d = w.B, w.Hq, w.NQ, w.NK, w.d
+    splits = binding.streamkl_fwd_splits(B, Hq, NQ, NK)
+    need = binding.streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, 0)
+    ws = torch.empty(max(4, need) // 4, dtype=torch.float32, device=dev)
+    out = tuple(torch.empty((B, Hq, NQ), device=dev) for _ in range(3))
+    stream = torch.cuda.current_stream()
+
+    def split():
+        binding.fwd_splitk(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal,
+                           splits=0, out=out, workspace=ws, stream=stream)
+
+    def unsplit():
+        binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal, out=out,
+                    stream=stream)
+
+    for _ in range(args.warmup):
+        split()
+        unsplit()
+    torch.cuda.synchronize()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
+
+    def timed(fn):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    s_ms = timed(split)
+    u_ms = timed(unsplit)
+    clk = clocks.stop()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
+    # algorithmic bytes: Q1, Q2, the keys once (shared), 12 bytes of output per row
+    rows = B * Hq * NQ
+    nbytes = 2 * rows * d * 2 + B * w.Hkv * NK * d * 2 * (1 if w.shared_k else 2) + 12 * rows
+    gbs = nbytes / (s_ms * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    line = {
+        "metric": "decode forward (split-K) GB/s of algorithmic HBM traffic", "value": gbs,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": s_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "B4 H32 NQ=1 NK=32768 d128 non-causal shared K (decode); step = "
+                               "split-K forward + merge",
+                   "splits": splits, "bytes_per_step": nbytes,
+                   "l2": "keys (1.07 GB) larger than the 126 MB L2; no flush"},
+        "unsplit_ms": u_ms, "speedup_vs_unsplit": u_ms / s_ms,
+        "roofline": {"bound": "hbm", "kernel": "streamkl_fwd_kernel (split) + merge",
+                     "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "peak_source": "%s hbm_gbs" % peak_src,
+                     "note": "achieved = algorithmic bytes per step / CUDA-event time of the step"},
+        "clocks": clk,
+        "gpu_launches": 2 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary
     (profiles/dram_traffic.txt, lines "<call> <bytes>"), or None."""
@@ -436,6 +522,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU-oracle baseline leg")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    ap.add_argument("--decode", action="store_true",
+                    help="measure the split-K forward on the decode workload instead of the step")
     ap.add_argument("--heads", type=int, default=32,
                     help="query/KV heads (32 = the headline workload; fewer only for profiler captures)")
     args = ap.parse_args()
@@ -443,6 +531,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode:
+        return run_decode(args)
     return run_gpu(args)
 
 

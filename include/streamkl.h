@@ -68,6 +68,42 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
                  float* kl, float* lse1, float* lse2, void* stream);
 
 /*
+ * Forward with the key tiles split into ranges, for few query rows and many keys (the
+ * decoding case the technical summary's "3. Otimizações de Kernel de GPU" names for split-K):
+ * each (query block, key range) is one CTA, so B*Hq*ceil(NQ/256) blocks that would leave
+ * most of the 148 SMs idle become enough CTAs to stream the keys at HBM speed.  Every range
+ * stores its rows' five running scalars; a second kernel merges the ranges exactly (each
+ * rescaled to the common maximum, the online recurrence's own correction) and writes the
+ * same outputs as streamkl_fwd.
+ *
+ *   splits    : number of key ranges; 0 = the library's choice (streamkl_fwd_splits).  A
+ *               value above the number of 128-key tiles is reduced to it, and ranges are
+ *               whole tiles, so fewer ranges than asked may be used.  1 = streamkl_fwd.
+ *   workspace : device buffer of at least streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ,
+ *               NK, splits) bytes, 16-byte aligned, owned by the caller; its contents on
+ *               entry do not matter.  May be NULL when that size is 0 (one range).
+ * Other arguments, outputs, errors and ownership as streamkl_fwd.  Two kernels are launched
+ * on `stream`; extra device memory: the workspace only.
+ */
+int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
+                        const uint16_t* k2, int B, int Hq, int Hkv, int NQ, int NK, int d,
+                        float scale, int causal, int splits, float* kl, float* lse1, float* lse2,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The number of key ranges streamkl_fwd_splitk uses for splits = 0: 1 when the query blocks
+ * alone fill the GPU, else the fewest ranges within 3 % of the best of a waves x (tiles per
+ * range + 2) model, at most 64.  Host-only; returns 1 for invalid sizes.
+ */
+int streamkl_fwd_splits(int B, int Hq, int NQ, int NK);
+
+/*
+ * Bytes of split-K workspace: 5 fp32 per query row per key range actually used (0 when only
+ * one range is used, or for invalid sizes).  splits = 0 means the library's choice.
+ */
+size_t streamkl_fwd_splitk_workspace_bytes(int B, int Hq, int NQ, int NK, int splits);
+
+/*
  * Bytes of fp32 workspace streamkl_bwd needs for these sizes: B*Hkv*ceil(NK/128)*128*d*4
  * (the dK accumulator, whole 128-row key tiles).  Returns 0 for sizes outside the supported
  * range.

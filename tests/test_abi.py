@@ -113,6 +113,46 @@ def test_bwd_rejects_on_host(lib, kw, want):
     assert bwd_call(_expect=want, **kw) == want
 
 
+def test_splitk_workspace_and_choice(lib):
+    # 5 fp32 per row per range actually used; ranges are whole 128-key tiles
+    assert binding.streamkl_fwd_splitk_workspace_bytes(2, 4, 1, 5000, 3) == 3 * 5 * 2 * 4 * 1 * 4
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 2, 1, 300, 64) == 3 * 5 * 2 * 4   # 3 tiles
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 1, 5, 1, 8) == 0                  # one tile
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 2, 1, 1000, 1) == 0
+    # 40 tiles in 6 ranges of 7 -> 6 used; in 7 ranges of 6 -> 7 used
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 1, 1, 5000, 6) == 6 * 5 * 4
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 1, 1, 5000, 7) == 7 * 5 * 4
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 1, 1, 1, -1) == 0
+    # the library's choice: none when the query blocks fill the GPU, several otherwise
+    assert binding.streamkl_fwd_splits(1, 32, 16384, 16384) == 1
+    assert binding.streamkl_fwd_splits(1, 1, 1, 128) == 1
+    s = binding.streamkl_fwd_splits(4, 32, 1, 32768)
+    assert 2 <= s <= 64
+    assert binding.streamkl_fwd_splitk_workspace_bytes(4, 32, 1, 32768, 0) == s * 5 * 4 * 32 * 4
+
+
+def splitk_call(**kw):
+    assert kw.pop("_expect") in HOST_REJECTIONS   # never reach a launch with fake pointers
+    args = dict(q1=FAKE, k1=FAKE, q2=FAKE, k2=FAKE, B=1, Hq=2, Hkv=1, NQ=1, NK=4096, d=128,
+                scale=0.088, causal=0, splits=4, kl=FAKE, lse1=FAKE, lse2=FAKE, workspace=FAKE,
+                workspace_bytes=4 * 5 * 2 * 4, stream=0)
+    args.update(kw)
+    return binding.streamkl_fwd_splitk(**args)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(splits=-1), binding.ERR_INVALID_ARG),
+    (dict(workspace=None), binding.ERR_INVALID_ARG),
+    (dict(workspace_bytes=4 * 5 * 2 * 4 - 4), binding.ERR_INVALID_ARG),
+    (dict(workspace=FAKE + 4), binding.ERR_UNSUPPORTED),
+    (dict(kl=None), binding.ERR_INVALID_ARG),
+    (dict(d=96), binding.ERR_UNSUPPORTED),
+    (dict(causal=1), binding.ERR_UNSUPPORTED),
+])
+def test_splitk_rejects_on_host(lib, kw, want):
+    assert splitk_call(_expect=want, **kw) == want
+
+
 def test_header_is_plain_c():
     """The public header compiles as C99 with no CUDA or torch headers."""
     import subprocess
