@@ -13,7 +13,8 @@
 // tiles past the diagonal are never loaded or multiplied.
 //
 // Roles (384 threads):  warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
-// warps 2-3 idle, warps 4-7 = statistics warpgroup of tile 0, warps 8-11 = tile 1.
+// warps 2-3 idle, warps 4-7 = statistics warpgroup of tile 0, warps 8-11 = tile 1 (when the
+// block has one query tile, the two warpgroups instead take alternate key tiles of it).
 // Warp w may touch TMEM lanes 32*(w%4) .. 32*(w%4)+31, so each statistics warp owns the
 // 32 rows that live in its lane quarter.
 //
@@ -40,6 +41,7 @@ struct FwdParams {
     float* kl;
     float* lse1;
     float* lse2;
+    int rep4;      // NQ <= 32: the query tile holds rows 0..31 in each 32-lane quarter
     int splits;    // key ranges per query block (1 = no split)
     int kps;       // key tiles per range
     float* part;   // splits > 1: partial state [splits][5][B*Hq*NQ]: m1, l1, m2, l2, acc
@@ -64,7 +66,8 @@ struct FwdCfg {
     static constexpr int S_FULL = 2 + 2 * kSlots;   // + t
     static constexpr int S_FREE = S_FULL + 2;       // + t
     static constexpr int DONE = S_FREE + 2;
-    static constexpr int kNumBars = DONE + 1;
+    static constexpr int MERGE = DONE + 1;          // partial states of a row are stored
+    static constexpr int kNumBars = MERGE + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;   // tmem address, abort flag
     static constexpr int kSmem = kMisc + 16 + 1024;     // + slack for 1024-byte alignment
 };
@@ -223,6 +226,12 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #pragma unroll
     for (int t = 0; t < 2; ++t) jend[t] = max(j0, min(nkt[t], j0 + p.kps));
     const int nj = max(jend[0], jend[1]);
+    // One query tile and at least two key tiles: the two TMEM halves and both statistics
+    // warpgroups take alternate key tiles of tile 0, so the MMAs of one key tile run while
+    // the other is folded.  Each row then has (alt ? 2 : 1) * (rep4 ? 4 : 1) partial states,
+    // merged in the CTA at the end.
+    const bool alt = (ntiles == 1) && (nj - j0 > 1);
+    const int n_contrib = (alt ? 2 : 1) * (p.rep4 ? 4 : 1);
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -236,6 +245,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             mbar_init(BAR(C::K_EMPTY + s), 1);
         }
         mbar_init(BAR(C::DONE), 1);
+        mbar_init(BAR(C::MERGE), alt ? 256 : 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -258,10 +268,13 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             for (int t = 0; t < ntiles; ++t) {
                 mbar_arrive_expect_tx(BAR(C::Q_FULL + t), 2 * C::kTile);
                 for (int bx = 0; bx < C::kBoxes; ++bx) {
-                    tma_load_3d(sb + C::kQ1 + t * C::kTile + bx * C::kBox, &tmQ1, BAR(C::Q_FULL + t),
-                                bx * 64, q0[t], bh);
-                    tma_load_3d(sb + C::kQ2 + t * C::kTile + bx * C::kBox, &tmQ2, BAR(C::Q_FULL + t),
-                                bx * 64, q0[t], bh);
+                    // rep4: four 32-row copies (4 KiB each; the swizzle pattern repeats every
+                    // 8 rows, so each copy sits exactly where rows 32c.. of a 128-row box go)
+                    for (int c = 0; c < (p.rep4 ? 4 : 1); ++c) {
+                        const uint32_t o = t * C::kTile + bx * C::kBox + c * 4096;
+                        tma_load_3d(sb + C::kQ1 + o, &tmQ1, BAR(C::Q_FULL + t), bx * 64, q0[t], bh);
+                        tma_load_3d(sb + C::kQ2 + o, &tmQ2, BAR(C::Q_FULL + t), bx * 64, q0[t], bh);
+                    }
                 }
             }
             uint32_t it = 0;
@@ -311,16 +324,26 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     ++it;
                 }
                 tc_fence_after();
-                for (int t = 0; t < ntiles; ++t) {
-                    if (j >= jend[t]) continue;
-                    if (j > j0) {
-                        if (!mbar_wait(BAR(C::S_FREE + t), (j - j0 - 1) & 1, abort_flag)) {
+                const int u = j - j0;
+                for (int t = 0; t < (alt ? 1 : ntiles); ++t) {
+                    // TMEM half h (= statistics warpgroup h) and how often it was used before
+                    int h, use;
+                    if (alt) {
+                        h = u & 1;
+                        use = u >> 1;
+                    } else {
+                        if (j >= jend[t]) continue;
+                        h = t;
+                        use = u;
+                    }
+                    if (use > 0) {
+                        if (!mbar_wait(BAR(C::S_FREE + h), (use - 1) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
-                    const uint32_t d1 = tmem + t * 256;
+                    const uint32_t d1 = tmem + h * 256;
                     const uint32_t d2 = d1 + 128;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
@@ -336,7 +359,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                                     sw128_desc(sb + C::kK + s2 * C::kTile + off, 16, 1024), idesc,
                                     k > 0);
                     }
-                    mma_commit(BAR(C::S_FULL + t));
+                    mma_commit(BAR(C::S_FULL + h));
                 }
                 mma_commit(BAR(C::K_EMPTY + s1));
                 if (!SHARED_K) mma_commit(BAR(C::K_EMPTY + s2));
@@ -347,40 +370,47 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         }
     } else if (warp >= 4) {
         // ================================================================ statistics
-        const int t = (warp - 4) >> 2;
+        const int g = (warp - 4) >> 2;          // warpgroup = TMEM half it reads
+        const int t = alt ? 0 : g;              // query tile whose rows it folds
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
-        if (t < ntiles) {
-            const int i = q0[t] + r;
-            const uint32_t tS1 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(t * 256);
+        const bool rep4 = p.rep4 != 0;
+        // rep4: every quarter holds rows 0..31, and warp `quarter` folds only key columns
+        // [32*quarter, 32*quarter + 32) of each tile; the four states are merged at the end
+        const int c_lo = rep4 ? quarter : 0;
+        const int c_hi = rep4 ? quarter + 1 : 4;
+        if (g < (alt ? 2 : ntiles)) {
+            const int i = q0[t] + (rep4 ? lane : r);
+            const uint32_t tS1 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * 256);
             const uint32_t tS2 = tS1 + 128;
             const float sl2 = p.sl2;
             float m1 = -1e30f, l1 = 0.f, m2 = -1e30f, l2 = 0.f, acc = 0.f;
             bool ok = true;
             // a warp whose 32 rows all lie past NQ only keeps the barrier protocol
-            const bool any_row = q0[t] + quarter * 32 < p.NQ;
-            for (int j = j0; j < jend[t]; ++j) {
-                if (!mbar_wait(BAR(C::S_FULL + t), (j - j0) & 1, abort_flag)) {
+            const bool any_row = rep4 || q0[t] + quarter * 32 < p.NQ;
+            for (int j = j0 + (alt ? g : 0); j < jend[t]; j += (alt ? 2 : 1)) {
+                const int use = alt ? (j - j0) >> 1 : j - j0;
+                if (!mbar_wait(BAR(C::S_FULL + g), use & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (!any_row) {
                     tc_fence_before();
-                    mbar_arrive(BAR(C::S_FREE + t));
+                    mbar_arrive(BAR(C::S_FREE + g));
                     continue;
                 }
                 const int kb = j * 128;
                 const bool masked = (kb + 128 > p.NK) || (p.causal && kb + 127 > q0[t]);
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = c_lo; c < c_hi; ++c) {
                     uint32_t xa[32], ya[32];
                     tmem_ld32(tS1 + c * 32, xa);
                     tmem_ld32(tS2 + c * 32, ya);
                     tmem_wait_ld();
-                    if (c == 3) {
+                    if (c == c_hi - 1) {
                         tc_fence_before();
-                        mbar_arrive(BAR(C::S_FREE + t));
+                        mbar_arrive(BAR(C::S_FREE + g));
                     }
                     if (!masked) {
                         fold_chunk_full(xa, ya, sl2, m1, l1, m2, l2, acc);
@@ -392,6 +422,39 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                                              : (lim <= 0 ? 0u : ((1u << lim) - 1u));
                         fold_chunk_masked(xa, ya, valid, sl2, m1, l1, m2, l2, acc);
                     }
+                }
+            }
+            if (n_contrib > 1) {
+                // The partial states of a row meet in key slot 0, reused only once every MMA
+                // has completed (hence every key copy has landed and been read), and one
+                // thread per row combines them like the split-K merge does.
+                ok = mbar_wait(BAR(C::DONE), 0, abort_flag) && ok;
+                float* mb = reinterpret_cast<float*>(smem + C::kK);
+                const int rows_per = rep4 ? 32 : 128;
+                const int rho = rep4 ? lane : r;
+                const int kappa = (alt ? g : 0) * (rep4 ? 4 : 1) + (rep4 ? quarter : 0);
+                const float st[5] = {m1, l1, m2, l2, acc};
+#pragma unroll
+                for (int f = 0; f < 5; ++f) mb[(kappa * 5 + f) * rows_per + rho] = st[f];
+                mbar_arrive(BAR(C::MERGE));
+                if (g == 0 && (!rep4 || quarter == 0)) {
+                    ok = mbar_wait(BAR(C::MERGE), 0, abort_flag) && ok;
+                    float M1 = -1e30f, M2 = -1e30f;
+                    for (int w = 0; w < n_contrib; ++w) {
+                        M1 = fmaxf(M1, mb[(w * 5 + 0) * rows_per + rho]);
+                        M2 = fmaxf(M2, mb[(w * 5 + 2) * rows_per + rho]);
+                    }
+                    float L1 = 0.f, L2 = 0.f, A = 0.f;
+                    for (int w = 0; w < n_contrib; ++w) {
+                        const float a1 = ex2(mb[(w * 5 + 0) * rows_per + rho] - M1);
+                        const float a2 = ex2(mb[(w * 5 + 2) * rows_per + rho] - M2);
+                        L1 = fmaf(mb[(w * 5 + 1) * rows_per + rho], a1, L1);
+                        A = fmaf(mb[(w * 5 + 4) * rows_per + rho], a1, A);
+                        L2 = fmaf(mb[(w * 5 + 3) * rows_per + rho], a2, L2);
+                    }
+                    m1 = M1; l1 = L1; m2 = M2; l2 = L2; acc = A;
+                } else {
+                    ok = false;   // one thread per row writes it
                 }
             }
             if (ok && i < p.NQ && p.splits > 1) {

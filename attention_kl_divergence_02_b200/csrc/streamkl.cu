@@ -44,9 +44,10 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view [planes, rows, d] of a dense bf16 tensor, 128-row x 64-column boxes, 128-byte
-// swizzle, zero fill outside the tensor.
-int make_map(CUtensorMap* map, const void* base, long long planes, long long rows, int d) {
+// 3-D view [planes, rows, d] of a dense bf16 tensor, box_rows-row x 64-column boxes
+// (128 rows unless asked), 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* map, const void* base, long long planes, long long rows, int d,
+             unsigned box_rows = 128) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
         snprintf(t_last_cuda_error, sizeof(t_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
@@ -54,7 +55,7 @@ int make_map(CUtensorMap* map, const void* base, long long planes, long long row
     }
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -199,11 +200,15 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
     const bool shared = (k1 == k2);
     CUtensorMap mq1, mq2, mk1, mk2;
     int rc;
-    if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d))) return rc;
-    if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d))) return rc;
+    // at most 32 query rows: they are loaded once into each 32-lane quarter of the query
+    // tile (32-row boxes), so that all four warps of a warpgroup can fold them
+    const int rep4 = NQ <= 32 ? 1 : 0;
+    if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d, rep4 ? 32 : 128))) return rc;
+    if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d, rep4 ? 32 : 128))) return rc;
     if ((rc = make_map(&mk1, k1, (long long)B * Hkv, NK, d))) return rc;
     if ((rc = make_map(&mk2, k2, (long long)B * Hkv, NK, d))) return rc;
     skl::FwdParams p;
+    p.rep4 = rep4;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NQ = NQ; p.NK = NK;
     p.causal = causal ? 1 : 0;
     p.n_qblk = (NQ + 255) / 256;
@@ -253,8 +258,10 @@ int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
     const long long blocks = (long long)B * Hq * ((NQ + 255) / 256);
     const int nkt = (NK + 127) / 128;
     if (blocks >= kNumSMs || nkt < 2) return 1;
-    // time model: waves of one CTA per SM, each CTA ~ its key tiles + 2 tiles of fixed cost
-    // (query load, pipeline fill and drain); the fewest ranges within 3 % of the best
+    // time model: waves of one CTA per SM, each CTA ~ its key tiles + 8 tiles of fixed cost
+    // (query load, pipeline fill and drain, partial store; 8 measured on B4 H32 NQ1 NK32768,
+    // where 128 blocks already fill the GPU and splitting lost 6 %); the fewest ranges within
+    // 3 % of the best
     double best = 1e300;
     int best_s = 1;
     std::vector<double> cost(65, 0.0);
@@ -263,7 +270,7 @@ int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
         split_ranges(NK, s, &kps, &used);
         const long long ctas = blocks * used;
         const double waves = (double)((ctas + kNumSMs - 1) / kNumSMs);
-        cost[s] = waves * (kps + 2);
+        cost[s] = waves * (kps + 8);
         if (cost[s] < best) best = cost[s];
     }
     for (int s = 1; s <= std::min(nkt, 64); ++s) {

@@ -66,9 +66,10 @@ WORKLOADS = {
                         note="B1 H32 N65536 d128 causal shared K; Q2 = Q1 + 0.5 N"),
     "gqa": Workload("gqa", 4, 32, 8, 2048, 32768, 64, False, False, (2,), 4, head_scaled=True,
                     note="B4 Hq32 Hkv8 NQ2048 NK32768 d64 non-causal distinct K; per-head Q scale U(0.5,2)"),
-    "decode": Workload("decode", 4, 32, 32, 1, 32768, 128, False, True, (), 5, 1.0, 0.5,
-                       note="B4 H32 NQ1 NK32768 d128 non-causal shared K (one query row per head "
-                            "against a long key sequence: the split-K forward); Q2 = Q1 + 0.5 N"),
+    "decode": Workload("decode", 1, 16, 16, 1, 131072, 128, False, True, (), 5, 1.0, 0.5,
+                       note="B1 H16 NQ1 NK131072 d128 non-causal shared K (one query row per head "
+                            "against a long key sequence: 16 query blocks for 148 SMs, the case "
+                            "the split-K forward is for); Q2 = Q1 + 0.5 N"),
 }
 
 

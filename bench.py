@@ -414,7 +414,7 @@ def run_gpu(args):
 
 
 def run_decode(args):
-    """Split-K forward on the decode workload (one query row per head, 32768 keys): bound by
+    """Split-K forward on the decode workload (one query row per head, 131072 keys): bound by
     streaming the keys from HBM, so it reports GB/s of algorithmic traffic against the
     measured copy bandwidth, and the unsplit forward beside it."""
     import torch
@@ -483,10 +483,10 @@ def run_decode(args):
         "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": s_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "B4 H32 NQ=1 NK=32768 d128 non-causal shared K (decode); step = "
-                               "split-K forward + merge",
+        "config": {"workload": "B1 H16 NQ=1 NK=131072 d128 non-causal shared K (decode); step "
+                               "= split-K forward + merge",
                    "splits": splits, "bytes_per_step": nbytes,
-                   "l2": "keys (1.07 GB) larger than the 126 MB L2; no flush"},
+                   "l2": "keys (537 MB) larger than the 126 MB L2; no flush"},
         "unsplit_ms": u_ms, "speedup_vs_unsplit": u_ms / s_ms,
         "roofline": {"bound": "hbm", "kernel": "streamkl_fwd_kernel (split) + merge",
                      "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,

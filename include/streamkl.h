@@ -93,7 +93,7 @@ int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* 
 /*
  * The number of key ranges streamkl_fwd_splitk uses for splits = 0: 1 when the query blocks
  * alone fill the GPU, else the fewest ranges within 3 % of the best of a waves x (tiles per
- * range + 2) model, at most 64.  Host-only; returns 1 for invalid sizes.
+ * range + 8) model, at most 64.  Host-only; returns 1 for invalid sizes.
  */
 int streamkl_fwd_splits(int B, int Hq, int NQ, int NK);
 

@@ -126,9 +126,10 @@ def test_splitk_workspace_and_choice(lib):
     # the library's choice: none when the query blocks fill the GPU, several otherwise
     assert binding.streamkl_fwd_splits(1, 32, 16384, 16384) == 1
     assert binding.streamkl_fwd_splits(1, 1, 1, 128) == 1
-    s = binding.streamkl_fwd_splits(4, 32, 1, 32768)
-    assert 2 <= s <= 64
-    assert binding.streamkl_fwd_splitk_workspace_bytes(4, 32, 1, 32768, 0) == s * 5 * 4 * 32 * 4
+    assert binding.streamkl_fwd_splits(4, 32, 1, 32768) == 1     # 128 blocks fill the GPU
+    s = binding.streamkl_fwd_splits(1, 16, 1, 131072)
+    assert 4 <= s <= 64
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 16, 1, 131072, 0) == s * 5 * 16 * 4
 
 
 def splitk_call(**kw):

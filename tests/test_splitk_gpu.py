@@ -1,7 +1,7 @@
 """Split-K forward (streamkl_fwd_splitk): the key tiles cut into ranges folded by separate
 CTAs, then merged exactly.  Checked through the C ABI against the fp64 oracle on the same
 seeded inputs, at small sizes that span several key ranges and ragged tiles, at the full
-decode workload (B4 H32 NQ=1 NK=32768 d128, every row), and against the unsplit forward."""
+decode workload (B1 H16 NQ=1 NK=131072 d128, every row), and against the unsplit forward."""
 import numpy as np
 import pytest
 import torch
@@ -60,7 +60,7 @@ def test_matches_unsplit_forward():
 
 def test_decode_workload_every_row():
     """Full decode workload in the configuration the benchmark times (library's choice of
-    ranges); the oracle computes all 128 rows."""
+    ranges); the oracle computes all 16 rows."""
     w = inputs.WORKLOADS["decode"]
     t = inputs.make(w, device="cuda")
     assert binding.streamkl_fwd_splits(w.B, w.Hq, w.NQ, w.NK) > 1
@@ -77,3 +77,18 @@ def test_workspace_too_small_is_refused_before_launch():
     rc = binding.streamkl_fwd_splitk(t["q1"], t["k1"], t["q2"], t["k2"], 1, 2, 2, 1, 4096, 128,
                                      w.scale, 0, 4, *out, ws, ws.numel() * 4)
     assert rc == binding.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("NQ,NK,causal,d", [(1, 1000, False, 128), (31, 777, False, 64),
+                                            (32, 4096, False, 128), (33, 500, False, 128),
+                                            (20, 20, True, 128), (7, 7, True, 64)])
+def test_few_rows_plain_forward(NQ, NK, causal, d):
+    """The unsplit forward at 32 query rows or fewer, where every warp of the warpgroup folds
+    a quarter of each key tile and the four partial states are merged in the CTA."""
+    w = inputs.custom(2, 2, 1, NQ, NK, d, causal, True, seed=100 + NQ)
+    t = inputs.make(w, device="cuda")
+    got = tuple(x.cpu().double().numpy()
+                for x in binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale,
+                                     causal=causal))
+    assert binding.streamkl_device_status() == binding.OK
+    check_fwd(got, _oracle(t, w), "few rows NQ=%d NK=%d" % (NQ, NK))
