@@ -57,6 +57,9 @@ struct BwdParams {
     const float* dkl;
     float* dk_ws;   // fp32, tile-blocked (see above)
     uint16_t* dq;   // bf16 [B,Hq,NQ,d]
+    int splits;     // key ranges per query tile (1 = one CTA sees all of a tile's keys)
+    int kps;        // key tiles per range
+    float* dq_ws;   // splits > 1: fp32 dQ partial sums, tile-blocked like dk_ws (planes B*Hq)
 };
 
 constexpr int kBwdThreads = 704;
@@ -97,22 +100,26 @@ struct BwdCfg {
     static constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDQ = 256, kColDK = 384;
 };
 
-// Visit n of a CTA -> key tile.  Causal: key tiles qt, qt-1, ..., 0 (diagonal first).
-// Non-causal: all key tiles, rotated by query tile and head so that CTAs working at the
-// same time reduce into different dK blocks.
+// Visit n of a CTA -> key tile.  The CTA owns key tiles [lo, hi): range `sp` of kps tiles,
+// clipped to the tiles its rows can see (causal: up to the diagonal tile qt).  Causal: from
+// the diagonal end downwards.  Non-causal: rotated by query tile and head so that CTAs
+// working at the same time reduce into different dK blocks.  count may be 0 (a range past
+// the diagonal).
 struct BwdSchedule {
-    int nkt, qt, rot, causal, count;
-    __device__ BwdSchedule(const BwdParams& p, int qt_, int h) {
-        nkt = p.nkt;
-        qt = qt_;
+    int lo, hi, rot, causal, count;
+    __device__ BwdSchedule(const BwdParams& p, int qt_, int h, int sp) {
         causal = p.causal;
-        rot = (qt_ + h) % p.nkt;
-        count = causal ? qt_ + 1 : p.nkt;
+        lo = sp * p.kps;
+        int end = min(p.nkt, lo + p.kps);
+        if (causal) end = min(end, qt_ + 1);
+        hi = end;
+        count = max(0, end - lo);
+        rot = count > 0 ? (qt_ + h) % count : 0;
     }
     __device__ int key_tile(int n) const {
-        if (causal) return qt - n;
+        if (causal) return hi - 1 - n;
         const int u = n + rot;
-        return u >= nkt ? u - nkt : u;
+        return lo + (u >= count ? u - count : u);
     }
 };
 
@@ -244,11 +251,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     // flight then reduce into the dK blocks of a few KV heads only (a few MB per head), so
     // the partial sums meet in L2 instead of going back and forth to DRAM (a group of 2
     // measured best of 2, 4, 8 and 16 on the causal and GQA workloads).
+    // With key ranges (few query tiles, many keys), the ranges of one query tile are
+    // neighbours in the grid.
     const int BH = p.B * p.Hq;
+    const int sp = blockIdx.x % p.splits;
+    const int ub = blockIdx.x / p.splits;
     const int per_group = kBwdHeadGroup * p.nqt;
-    const int group = blockIdx.x / per_group;
+    const int group = ub / per_group;
     const int gh = min(kBwdHeadGroup, BH - group * kBwdHeadGroup);   // planes in this group
-    const int r_in = blockIdx.x - group * per_group;
+    const int r_in = ub - group * per_group;
     const int unit = r_in / gh;
     const int bh = group * kBwdHeadGroup + r_in % gh;
     const int qt = p.causal ? (p.nqt - 1 - unit) : unit;
@@ -256,7 +267,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int h = bh % p.Hq;
     const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
     const int q0 = qt * 128;
-    const BwdSchedule sched(p, qt, h);
+    const BwdSchedule sched(p, qt, h, sp);
     const int N = sched.count;
     constexpr bool mode1 = (MODE == 1);
     // Key tiles of a visit enter the ring in the order (fixed distribution's, free
@@ -374,7 +385,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 return true;
             };
             bool ok = mbar_wait(BAR(C::Q_FULL), 0, abort_flag);
-            if (ok) ok = issue_S(0);
+            if (ok && N > 0) ok = issue_S(0);
             for (int n = 0; n < N && ok; ++n) {
                 if (n + 1 < N) {
                     if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
@@ -521,8 +532,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             fence_async_smem();
             mbar_arrive(BAR(C::DS_FULL + (n & 1)));
         }
-        // dQ of this query tile, accumulated over every visit: scale, round, store
-        if (ok && mbar_wait(BAR(C::DQ_DONE), 0, abort_flag)) {
+        // dQ of this query tile, accumulated over every visit of the CTA.  One key range:
+        // scale, round, store.  Several: add it into the fp32 dQ workspace (the convert kernel
+        // scales and rounds once every range has added its part).
+        if (ok && N > 0 && mbar_wait(BAR(C::DQ_DONE), 0, abort_flag)) {
             tc_fence_after();
             constexpr int kCols = D / 4;          // dQ columns per warpgroup
             uint32_t v[kCols];
@@ -532,7 +545,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 tmem_ld16(lane_base + C::kColDQ + wg * kCols, v);
             }
             tmem_wait_ld();
-            if (q < p.NQ) {
+            if (p.splits > 1) {
+                // tile-blocked: [quarter][32-column chunk][4-column group][lane][4]
+                float* blk = p.dq_ws + ((size_t)bh * p.nqt + qt) * (128 * D) +
+                             (size_t)quarter * (32 * D) + lane * 4;
+                const int c = (wg * kCols) / 32;          // chunk of this warpgroup's columns
+                const int g0 = ((wg * kCols) % 32) / 4;   // first 4-column group in the chunk
+#pragma unroll
+                for (int g = 0; g < kCols / 4; ++g)
+                    red_add_v4(blk + c * 1024 + (g0 + g) * 128, v[4 * g], v[4 * g + 1], v[4 * g + 2],
+                               v[4 * g + 3]);
+            } else if (q < p.NQ) {
                 uint4* dst = reinterpret_cast<uint4*>(p.dq + ((size_t)bh * p.NQ + q) * D + wg * kCols);
 #pragma unroll
                 for (int k = 0; k < kCols / 8; ++k) {

@@ -101,6 +101,20 @@ int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
     return STREAMKL_OK;
 }
 
+// fp32 tile-blocked workspace -> bf16 rows (scale applied), one launch.
+template <int D>
+int launch_convert(const float* ws, uint16_t* out, int planes, int rows, int ntiles, float scale,
+                   cudaStream_t st, const char* what) {
+    const size_t threads = (size_t)planes * ntiles * 128 * (D / 32);
+    size_t blocks = (threads + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    skl::streamkl_tile_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(ws, out, planes, rows, ntiles,
+                                                                          scale);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return STREAMKL_OK;
+}
+
 template <int D, bool SHARED>
 int launch_bwd(int mode, const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                const CUtensorMap& k2, const skl::BwdParams& p, int grid, size_t ws_bytes,
@@ -114,14 +128,9 @@ int launch_bwd(int mode, const CUtensorMap& q1, const CUtensorMap& q2, const CUt
     kern<<<grid, skl::kBwdThreads, smem, st>>>(q1, q2, k1, k2, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_bwd launch");
-    const size_t threads = (size_t)p.B * p.Hkv * p.nkt * 128 * (D / 32);
-    size_t blocks = (threads + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    skl::streamkl_tile_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(p.dk_ws, dk, p.B * p.Hkv,
-                                                                          p.NK, p.nkt, p.scale);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dk convert launch");
-    return STREAMKL_OK;
+    rc = launch_convert<D>(p.dk_ws, dk, p.B * p.Hkv, p.NK, p.nkt, p.scale, st, "dk convert launch");
+    if (rc || p.splits == 1) return rc;
+    return launch_convert<D>(p.dq_ws, p.dq, p.B * p.Hq, p.NQ, p.nqt, p.scale, st, "dq convert launch");
 }
 
 }  // namespace
@@ -310,10 +319,51 @@ int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* 
                     static_cast<float*>(workspace), stream);
 }
 
-size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d) {
-    if (B < 1 || Hq < 1 || Hkv < 1 || NQ < 1 || NK < 1 || (d != 64 && d != 128)) return 0;
+}  // extern "C"
+
+namespace {
+
+// Key ranges per query tile for the backward: 1 when the query tiles fill the GPU, else the
+// fewest ranges within 3 % of the best of a waves x (tiles per range + 6) model (6 tiles of
+// fixed cost per CTA: query load, pipeline fill, dQ reduction), at most 32.
+int bwd_splits(int B, int Hq, int NQ, int NK) {
+    const long long ctas = (long long)B * Hq * ((NQ + 127) / 128);
+    const int nkt = (NK + 127) / 128;
+    if (ctas >= kNumSMs || nkt < 2) return 1;
+    double cost[33] = {0};
+    double best = 1e300;
+    for (int s = 1; s <= std::min(nkt, 32); ++s) {
+        int kps, used;
+        split_ranges(NK, s, &kps, &used);
+        const double waves = (double)((ctas * used + kNumSMs - 1) / kNumSMs);
+        cost[s] = waves * (kps + 6);
+        best = std::min(best, cost[s]);
+    }
+    for (int s = 1; s <= std::min(nkt, 32); ++s) {
+        if (cost[s] <= best * 1.03) {
+            int kps, used;
+            split_ranges(NK, s, &kps, &used);
+            return used;
+        }
+    }
+    return 1;
+}
+
+size_t bwd_dk_bytes(int B, int Hkv, int NK, int d) {
     const size_t rows = (size_t)(NK + 127) / 128 * 128;   // whole 128-row key tiles
     return (size_t)B * Hkv * rows * d * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || NQ < 1 || NK < 1 || (d != 64 && d != 128)) return 0;
+    size_t bytes = bwd_dk_bytes(B, Hkv, NK, d);
+    if (bwd_splits(B, Hq, NQ, NK) > 1)   // plus the dQ partial sums, tile-blocked
+        bytes += (size_t)B * Hq * ((NQ + 127) / 128 * 128) * d * sizeof(float);
+    return bytes;
 }
 
 int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_t* q2,
@@ -346,7 +396,14 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
     p.kl = kl; p.lse1 = lse1; p.lse2 = lse2; p.dkl = dkl;
     p.dk_ws = static_cast<float*>(workspace);
     p.dq = dq;
-    const long long grid = (long long)B * Hq * p.nqt;
+    p.splits = bwd_splits(B, Hq, NQ, NK);
+    {
+        int used;
+        split_ranges(NK, p.splits, &p.kps, &used);
+        p.splits = used;
+    }
+    p.dq_ws = p.splits > 1 ? p.dk_ws + bwd_dk_bytes(B, Hkv, NK, d) / sizeof(float) : nullptr;
+    const long long grid = (long long)B * Hq * p.nqt * p.splits;
     if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
     const size_t ws = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -66,6 +66,10 @@ WORKLOADS = {
                         note="B1 H32 N65536 d128 causal shared K; Q2 = Q1 + 0.5 N"),
     "gqa": Workload("gqa", 4, 32, 8, 2048, 32768, 64, False, False, (2,), 4, head_scaled=True,
                     note="B4 Hq32 Hkv8 NQ2048 NK32768 d64 non-causal distinct K; per-head Q scale U(0.5,2)"),
+    "chunk": Workload("chunk", 1, 16, 16, 512, 65536, 128, False, True, (1, 2), 6, 1.0, 0.5,
+                      note="B1 H16 NQ512 NK65536 d128 non-causal shared K (a chunk of queries "
+                           "against a long context: 64 query tiles for 148 SMs, the case the "
+                           "key-range backward is for); Q2 = Q1 + 0.5 N"),
     "decode": Workload("decode", 1, 16, 16, 1, 131072, 128, False, True, (), 5, 1.0, 0.5,
                        note="B1 H16 NQ1 NK131072 d128 non-causal shared K (one query row per head "
                             "against a long key sequence: 16 query blocks for 148 SMs, the case "

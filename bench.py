@@ -499,6 +499,89 @@ def run_decode(args):
     return 0
 
 
+def run_chunk(args):
+    """Backward (both settings) on the chunk workload (512 query rows per head against 65536
+    keys): 64 query tiles for 148 SMs, so the library splits every tile's keys into ranges.
+    Reports TFLOP/s of the backward against the measured tensor peak."""
+    import torch
+
+    from attention_kl_divergence_02_b200 import binding, inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--chunk measures one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    binding.load()
+    w = inputs.WORKLOADS["chunk"]
+    t = inputs.make(w, device=dev)
+    B, Hq, NQ, NK, d = w.B, w.Hq, w.NQ, w.NK, w.d
+    stream = torch.cuda.current_stream()
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, stream=stream)
+    ws_bytes = binding.streamkl_bwd_workspace_bytes(B, Hq, w.Hkv, NQ, NK, d)
+    dk_part = B * w.Hkv * ((NK + 127) // 128 * 128) * d * 4
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
+    g = (torch.empty_like(t["q1"]), torch.empty_like(t["k1"]))
+
+    def bwd(mode):
+        binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], scale=w.scale,
+                    out=g, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        bwd(1)
+        bwd(2)
+    torch.cuda.synchronize()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
+
+    def timed(mode):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            bwd(mode)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    m1 = timed(1)
+    m2 = timed(2)
+    clk = clocks.stop()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
+    flops = w.bwd_flops()
+    t1, t2 = flops / (m1 * 1e-3) / 1e12, flops / (m2 * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = {
+        "metric": "backward TFLOP/s, query chunk against a long context (key-range backward)",
+        "value": 2 * flops / ((m1 + m2) * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m1 + m2,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "B1 H16 NQ=512 NK=65536 d128 non-causal shared K (chunk); step = "
+                               "backward P1-fixed + backward P2-fixed",
+                   "key_ranges_in_use": ws_bytes > dk_part,
+                   "l2": "inputs and dK workspace (0.54 GB) larger than the 126 MB L2; no flush"},
+        "bwd_mode1_ms": m1, "bwd_mode1_tflops": t1, "bwd_mode2_ms": m2, "bwd_mode2_tflops": t2,
+        "roofline": {"bound": "tensor", "kernel": "bwd_mode1", "achieved": t1, "peak": peak,
+                     "unit": "TFLOP/s", "frac": t1 / peak, "traffic": None,
+                     "peak_source": "%s bf16_tflops (burst)" % peak_src,
+                     "note": "achieved = algorithmic FLOPs (8d per pair) / CUDA-event time of the "
+                             "call (memset, kernel, dK and dQ converts)"},
+        "clocks": clk,
+        "gpu_launches": 3 * 2 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary
     (profiles/dram_traffic.txt, lines "<call> <bytes>"), or None."""
@@ -524,6 +607,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
     ap.add_argument("--decode", action="store_true",
                     help="measure the split-K forward on the decode workload instead of the step")
+    ap.add_argument("--chunk", action="store_true",
+                    help="measure the key-range backward on the chunk workload instead of the step")
     ap.add_argument("--heads", type=int, default=32,
                     help="query/KV heads (32 = the headline workload; fewer only for profiler captures)")
     args = ap.parse_args()
@@ -533,6 +618,8 @@ def main():
         return run_reference(args)
     if args.decode:
         return run_decode(args)
+    if args.chunk:
+        return run_chunk(args)
     return run_gpu(args)
 
 

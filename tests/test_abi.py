@@ -44,11 +44,15 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_bytes(lib):
-    # the dK accumulator: B * Hkv * whole 128-row key tiles * d fp32
+    # the dK accumulator: B * Hkv * whole 128-row key tiles * d fp32 ...
     assert binding.streamkl_bwd_workspace_bytes(1, 32, 32, 16384, 16384, 128) == 32 * 16384 * 128 * 4
     assert binding.streamkl_bwd_workspace_bytes(2, 6, 3, 5, 5, 64) == 2 * 3 * 128 * 64 * 4
-    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 7, 129, 128) == 256 * 128 * 4
     assert binding.streamkl_bwd_workspace_bytes(4, 32, 8, 2048, 32768, 64) == 4 * 8 * 32768 * 64 * 4
+    # ... plus, when the query tiles alone would leave SMs idle and their keys are split into
+    # ranges, the dQ partial sums: B * Hq * whole 128-row query tiles * d fp32
+    assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 7, 129, 128) == 256 * 128 * 4 + 128 * 128 * 4
+    assert binding.streamkl_bwd_workspace_bytes(1, 16, 16, 512, 65536, 128) == (
+        16 * 65536 * 128 * 4 + 16 * 512 * 128 * 4)
     assert binding.streamkl_bwd_workspace_bytes(1, 1, 1, 1, 1, 96) == 0
     assert binding.streamkl_bwd_workspace_bytes(0, 1, 1, 1, 1, 64) == 0
 
