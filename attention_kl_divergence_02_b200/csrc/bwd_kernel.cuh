@@ -357,6 +357,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             constexpr uint32_t idK = idesc_bf16(128, D, 1, 1);     // dS^T MN-major, Q MN-major
             auto slot_of = [&](int n, int j) { return (uint32_t)(ring_idx(n, j) % C::kSlots); };
             auto fill_parity = [&](int n, int j) { return (uint32_t)((ring_idx(n, j) / C::kSlots) & 1); };
+            // Descriptors are built once per operand base and advanced by the operand's byte
+            // offset / 16 (the 14-bit start-address field cannot carry: shared addresses stay
+            // below 2^18 and every offset is a multiple of 16), so the issuing thread spends
+            // about one instruction per descriptor between MMAs; those of the resident query
+            // tiles are loop-invariant.
+            auto dadd = [](uint64_t dsc, uint32_t bytes) { return dsc + (uint64_t)(bytes >> 4); };
+            const uint64_t dq1k = sw128_desc(sb + C::kQ1, 16, 1024);        // Q1, K-major
+            const uint64_t dq2k = sw128_desc(sb + C::kQ2, 16, 1024);        // Q2, K-major
+            const uint64_t dqfm = sw128_desc(qfree, C::kBox, 1024);         // Q_free, MN-major
             // S of visit n; returns false if a wait gave up
             auto issue_S = [&](int n) -> bool {
                 const uint32_t s1 = slot_of(n, kJ1);
@@ -365,19 +374,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 if (!SHARED_K && !mbar_wait(BAR(C::K_FULL + s2), fill_parity(n, kJ2), abort_flag))
                     return false;
                 tc_fence_after();
-                const uint32_t k1s = sb + C::kRing + s1 * C::kTile;
-                const uint32_t k2s = sb + C::kRing + s2 * C::kTile;
+                const uint64_t dk1 = sw128_desc(sb + C::kRing + s1 * C::kTile, 16, 1024);
+                const uint64_t dk2 = SHARED_K ? dk1 : sw128_desc(sb + C::kRing + s2 * C::kTile, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS1, sw128_desc(sb + C::kQ1 + off, 16, 1024),
-                                sw128_desc(k1s + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS1, dadd(dq1k, off), dadd(dk1, off), idS, k > 0);
                 }
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS2, sw128_desc(sb + C::kQ2 + off, 16, 1024),
-                                sw128_desc(k2s + off, 16, 1024), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS2, dadd(dq2k, off), dadd(dk2, off), idS, k > 0);
                 }
                 mma_commit(BAR(C::S_FULL));
                 // with distinct keys, the fixed distribution's key tile (j = 0) is done after S
@@ -393,22 +400,24 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     if (!issue_S(n + 1)) break;
                 }
                 const uint32_t ds = sb + C::kDS + (n & 1) * C::kDSBuf;
+                const uint64_t ddsk = sw128_desc(ds, 16, 1024);         // dS, K-major (A of dQ)
+                const uint64_t ddsm = sw128_desc(ds, C::kBox, 1024);    // dS^T, MN-major (A of dK)
+                const uint64_t dkfm = sw128_desc(sb + C::kRing + slot_of(n, kJFree) * C::kTile,
+                                                 C::kBox, 1024);        // K_free, MN-major
                 if (!mbar_wait(BAR(C::DS_FULL + (n & 1)), (n >> 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 // dQ += dS K_free, accumulated over every visit; it does not wait for the flush
-                const uint32_t kf = sb + C::kRing + slot_of(n, kJFree) * C::kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDQ,
-                                sw128_desc(ds + (k >> 2) * C::kBox + (k & 3) * 32, 16, 1024),
-                                sw128_desc(kf + k * 2048, C::kBox, 1024), idQ, (n > 0 || k > 0));
+                    mma_bf16_ss(tmem + C::kColDQ, dadd(ddsk, (k >> 2) * C::kBox + (k & 3) * 32),
+                                dadd(dkfm, k * 2048), idQ, (n > 0 || k > 0));
                 }
                 mma_commit(BAR(C::K_EMPTY + slot_of(n, kJFree)));
                 // dK partial of this key tile: dS^T Q_free (fresh every visit)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDK, sw128_desc(ds + k * 2048, C::kBox, 1024),
-                                sw128_desc(qfree + k * 2048, C::kBox, 1024), idK, k > 0);
+                    mma_bf16_ss(tmem + C::kColDK, dadd(ddsm, k * 2048), dadd(dqfm, k * 2048), idK,
+                                k > 0);
                 }
                 mma_commit(BAR(C::DK_FULL));
                 mma_commit(BAR(C::DS_FREE + (n & 1)));
