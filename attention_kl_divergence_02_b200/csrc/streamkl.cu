@@ -183,7 +183,7 @@ int streamkl_selftest_watchdog(int starve, long long* waited_ns, void* stream) {
         waited_ns[0] = (long long)res[1];
         waited_ns[1] = (long long)res[2];
     }
-    // both waits must agree with the verdict: all passed (OK) or none did (TIMEOUT)
+    // both waits must agree with the status: all passed (OK) or none did (TIMEOUT)
     if (status == STREAMKL_OK && res[0] != 3ull) return STREAMKL_ERR_TIMEOUT;
     if (status != STREAMKL_OK && res[0] != 0ull) return STREAMKL_ERR_CUDA;
     return status;

@@ -18,6 +18,7 @@ import json
 import math
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -89,7 +90,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+        self.path = os.path.join(tempfile.gettempdir(), "streamkl_clocks_rank%d.csv" % gpu_index)
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
