@@ -158,3 +158,42 @@ def test_full_size_headline(mode):
 
 def test_full_size_gqa_mode2():
     sampled_check("gqa", 2, heads_for_dk=1, rows_per_head=16, keys_per_head=32)
+
+
+SIGN_CASES = [
+    # B, Hq, Hkv, NQ, NK, d, causal, shared
+    (1, 2, 2, 300, 700, 128, False, False),
+    (1, 1, 1, 640, 640, 128, True, True),      # key ranges per query tile (few query tiles)
+    (2, 4, 2, 129, 260, 64, False, True),
+]
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("kind", ["signed", "zeros"])
+@pytest.mark.parametrize("case", SIGN_CASES, ids=lambda c: "NQ%dNK%dd%d%s" % (c[3], c[4], c[5], "c" if c[6] else ""))
+def test_upstream_gradient_signs_and_zeros(case, kind, mode):
+    """g of both signs takes the path that multiplies by g (a warp with any g < 0 cannot fold
+    log2 g into the exponent); g = 0 on every third row exercises the folded path's
+    log2 0 = -inf, which must leave those rows' dQ negligible: the exponential unit gives
+    exactly 0 there, the FMA-pipe exp2 (which clamps its argument at -126 to stay finite)
+    2^-126, so a zero row's dQ is at most of order 1e-36."""
+    B, Hq, Hkv, NQ, NK, d, causal, shared = case
+    w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=NQ + NK + d + 1)
+    t = inputs.make(w, device="cuda")
+    gen = torch.Generator().manual_seed(17)
+    if kind == "signed":
+        g = torch.randn(t["dkl"].shape, generator=gen)
+    else:
+        g = torch.rand(t["dkl"].shape, generator=gen) + 0.25
+        g[..., ::3] = 0.0
+    t["dkl"] = g.cuda()
+    dq, dk = gpu_bwd(t, w, mode)
+    h = host(t)
+    odq, odk = oracle.bwd(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], scale=w.scale,
+                          causal=w.causal)
+    zero_atol = 1e-6 * w.scale * float(np.abs(h["dkl"]).max()) * max(np.abs(h["q1"]).max(), np.abs(h["q2"]).max()) \
+        * max(np.abs(h["k1"]).max(), np.abs(h["k2"]).max())
+    check_grad(dq, odq, "%s %s dQ mode %d" % (case, kind, mode), zero_atol)
+    check_grad(dk, odk, "%s %s dK mode %d" % (case, kind, mode), zero_atol)
+    if kind == "zeros":
+        assert np.abs(dq[..., ::3, :]).max() <= 1e-30
