@@ -232,20 +232,25 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     // merged in the CTA at the end.
     const bool alt = (ntiles == 1) && (nj - j0 > 1);
     const int n_contrib = (alt ? 2 : 1) * (p.rep4 ? 4 : 1);
+    // Two query tiles: warpgroup g folds key columns [64g, 64g + 64) of BOTH tiles (a thread
+    // can read its row in either tile's TMEM columns).  Tile t's S is then free as soon as
+    // both warpgroups have loaded their two chunks of it, and its next MMAs run while the
+    // warpgroups fold the other tile.  The two column halves of a row merge at the end.
+    const bool split = (ntiles == 2);
 
     // ---- setup
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             mbar_init(BAR(C::Q_FULL + t), 1);
             mbar_init(BAR(C::S_FULL + t), 1);
-            mbar_init(BAR(C::S_FREE + t), 128);
+            mbar_init(BAR(C::S_FREE + t), split ? 256 : 128);
         }
         for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(BAR(C::K_FULL + s), 1);
             mbar_init(BAR(C::K_EMPTY + s), 1);
         }
         mbar_init(BAR(C::DONE), 1);
-        mbar_init(BAR(C::MERGE), alt ? 256 : 128);
+        mbar_init(BAR(C::MERGE), (alt || split) ? 256 : 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -379,7 +384,105 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         // [32*quarter, 32*quarter + 32) of each tile; the four states are merged at the end
         const int c_lo = rep4 ? quarter : 0;
         const int c_hi = rep4 ? quarter + 1 : 4;
-        if (g < (alt ? 2 : ntiles)) {
+        // writes one finished row: its partial state (split-K) or KL, LSE1, LSE2
+        auto write_row = [&](int i, float m1, float l1, float m2, float l2, float acc) {
+            if (p.splits > 1) {
+                const size_t R = (size_t)p.B * p.Hq * p.NQ;
+                float* dst = p.part + (size_t)sp * 5 * R + (size_t)bh * p.NQ + i;
+                dst[0] = m1;
+                dst[R] = l1;
+                dst[2 * R] = m2;
+                dst[3 * R] = l2;
+                dst[4 * R] = acc;
+            } else {
+                const float LN2 = 0.6931471805599453f;
+                const float lg1 = log2f(l1);
+                const float lg2 = log2f(l2);
+                const size_t o = (size_t)bh * p.NQ + i;
+                p.lse1[o] = (m1 + lg1) * LN2;
+                p.lse2[o] = (m2 + lg2) * LN2;
+                p.kl[o] = p.scale * acc / l1 + ((m2 - m1) + (lg2 - lg1)) * LN2;
+            }
+        };
+        if (split && g < 2) {
+            const float sl2 = p.sl2;
+            const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+            float st[2][5];
+#pragma unroll
+            for (int t2 = 0; t2 < 2; ++t2) {
+                st[t2][0] = -1e30f; st[t2][1] = 0.f; st[t2][2] = -1e30f; st[t2][3] = 0.f; st[t2][4] = 0.f;
+            }
+            bool ok = true;
+            for (int j = j0; j < nj && ok; ++j) {
+#pragma unroll
+                for (int t2 = 0; t2 < 2; ++t2) {
+                    if (!ok || j >= jend[t2]) continue;
+                    if (!mbar_wait(BAR(C::S_FULL + t2), (j - j0) & 1, abort_flag)) {
+                        ok = false;
+                        continue;
+                    }
+                    tc_fence_after();
+                    if (q0[t2] + quarter * 32 >= p.NQ) {   // no valid row in this warp
+                        tc_fence_before();
+                        mbar_arrive(BAR(C::S_FREE + t2));
+                        continue;
+                    }
+                    const int i2 = q0[t2] + r;
+                    const uint32_t tS1 = tmem + lanes + (uint32_t)(t2 * 256);
+                    const uint32_t tS2 = tS1 + 128;
+                    const int kb = j * 128;
+                    const bool masked = (kb + 128 > p.NK) || (p.causal && kb + 127 > q0[t2]);
+#pragma unroll 1
+                    for (int c = 2 * g; c < 2 * g + 2; ++c) {
+                        uint32_t xa[32], ya[32];
+                        tmem_ld32(tS1 + c * 32, xa);
+                        tmem_ld32(tS2 + c * 32, ya);
+                        tmem_wait_ld();
+                        if (c == 2 * g + 1) {
+                            tc_fence_before();
+                            mbar_arrive(BAR(C::S_FREE + t2));
+                        }
+                        if (!masked) {
+                            fold_chunk_full(xa, ya, sl2, st[t2][0], st[t2][1], st[t2][2], st[t2][3], st[t2][4]);
+                        } else {
+                            const int k0 = kb + c * 32;
+                            int lim = p.NK - k0;
+                            if (p.causal) lim = min(lim, i2 - k0 + 1);
+                            const uint32_t valid = lim >= 32 ? 0xFFFFFFFFu
+                                                 : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+                            fold_chunk_masked(xa, ya, valid, sl2, st[t2][0], st[t2][1], st[t2][2],
+                                              st[t2][3], st[t2][4]);
+                        }
+                    }
+                }
+            }
+            // the two column halves of every row meet in key slot 0 once every MMA (hence
+            // every key copy) is complete; warpgroup 0 combines them and writes both tiles
+            ok = mbar_wait(BAR(C::DONE), 0, abort_flag) && ok;
+            float* mb = reinterpret_cast<float*>(smem + C::kK);
+#pragma unroll
+            for (int t2 = 0; t2 < 2; ++t2)
+#pragma unroll
+                for (int f = 0; f < 5; ++f) mb[((t2 * 2 + g) * 5 + f) * 128 + r] = st[t2][f];
+            mbar_arrive(BAR(C::MERGE));
+            if (g == 0) {
+                ok = mbar_wait(BAR(C::MERGE), 0, abort_flag) && ok;
+#pragma unroll
+                for (int t2 = 0; t2 < 2; ++t2) {
+                    const float* a0 = mb + (t2 * 2 + 0) * 5 * 128 + r;
+                    const float* a1 = mb + (t2 * 2 + 1) * 5 * 128 + r;
+                    const float M1 = fmaxf(a0[0], a1[0]);
+                    const float M2 = fmaxf(a0[2 * 128], a1[2 * 128]);
+                    const float e10 = ex2(a0[0] - M1), e11 = ex2(a1[0] - M1);
+                    const float e20 = ex2(a0[2 * 128] - M2), e21 = ex2(a1[2 * 128] - M2);
+                    const float L1 = fmaf(a0[128], e10, a1[128] * e11);
+                    const float A = fmaf(a0[4 * 128], e10, a1[4 * 128] * e11);
+                    const float L2 = fmaf(a0[3 * 128], e20, a1[3 * 128] * e21);
+                    const int i2 = q0[t2] + r;
+                    if (ok && i2 < p.NQ) write_row(i2, M1, L1, M2, L2, A);
+                }
+            }
+        } else if (!split && g < (alt ? 2 : ntiles)) {
             const int i = q0[t] + (rep4 ? lane : r);
             const uint32_t tS1 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * 256);
             const uint32_t tS2 = tS1 + 128;
@@ -457,23 +560,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     ok = false;   // one thread per row writes it
                 }
             }
-            if (ok && i < p.NQ && p.splits > 1) {
-                const size_t R = (size_t)p.B * p.Hq * p.NQ;
-                float* dst = p.part + (size_t)sp * 5 * R + (size_t)bh * p.NQ + i;
-                dst[0] = m1;
-                dst[R] = l1;
-                dst[2 * R] = m2;
-                dst[3 * R] = l2;
-                dst[4 * R] = acc;
-            } else if (ok && i < p.NQ) {
-                const float LN2 = 0.6931471805599453f;
-                const float lg1 = log2f(l1);
-                const float lg2 = log2f(l2);
-                const size_t o = (size_t)bh * p.NQ + i;
-                p.lse1[o] = (m1 + lg1) * LN2;
-                p.lse2[o] = (m2 + lg2) * LN2;
-                p.kl[o] = p.scale * acc / l1 + ((m2 - m1) + (lg2 - lg1)) * LN2;
-            }
+            if (ok && i < p.NQ) write_row(i, m1, l1, m2, l2, acc);
         }
     }
 
