@@ -398,6 +398,9 @@ def run_gpu(args):
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # the calls are timed inside a step repeated back to back under the power cap: the
+    # roofline takes the sustained GEMM figure, the burst one is reported beside it
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     calls = {"fwd": (f_ms, w.fwd_flops()), "bwd_mode1": (b1_ms, w.bwd_flops()),
              "bwd_mode2": (b2_ms, w.bwd_flops())}
     dom = max(calls, key=lambda k: calls[k][0])
@@ -424,9 +427,11 @@ def run_gpu(args):
                         "basis": "%s bf16 %.1f TFLOP/s (burst); nominal dense %.0f gives fwd %.1f%%"
                                  % (peak_src, peak, NOMINAL_BF16_TFLOPS,
                                     100 * w.fwd_flops() / (f_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS)},
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": "%s bf16_tflops (burst)" % peak_src,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                     "peak_source": "%s bf16_tflops_sustained (timed inside a step repeated "
+                                    "back to back)" % peak_src,
+                     "peak_burst": peak, "frac_of_burst": achieved / peak,
                      "note": "achieved = algorithmic FLOPs per call / CUDA-event duration of the "
                              "call on its stream%s" % (
                                  "; the backward call also runs the dQ-workspace memset and the "
