@@ -138,3 +138,14 @@ def test_full_size_sampled(name):
         got = tuple(x.reshape(-1)[rows] for x in (kl, l1, l2))
         check_fwd(got, want, "%s causal=%s" % (name, causal))
         assert np.all(kl >= -2e-3)
+
+
+def test_reverse_kl_by_swapping_the_distributions():
+    """KL(P2||P1) through the same call with the two distributions' arguments swapped."""
+    w = inputs.custom(1, 2, 2, 300, 300, 128, True, False, seed=41)
+    t = inputs.make(w, device="cuda")
+    got = binding.fwd(t["q2"], t["k2"], t["q1"], t["k1"], scale=w.scale, causal=True)
+    assert binding.streamkl_device_status() == binding.OK
+    want = oracle.fwd(host64(t["q2"]), host64(t["k2"]), host64(t["q1"]), host64(t["k1"]),
+                      scale=w.scale, causal=True)
+    check_fwd(tuple(x.cpu().double().numpy() for x in got), want, "reverse KL")

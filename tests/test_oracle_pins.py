@@ -199,6 +199,26 @@ def test_kl_nonnegative_and_zero_on_identity():
         assert np.all(kl0 == 0.0) and np.array_equal(a, b)
 
 
+def test_reverse_and_symmetric_kl_against_brute_force():
+    """Swapping the two distributions' arguments gives KL(P2||P1); the sum of both
+    directions equals sum_j (p1 - p2)(log p1 - log p2), computed here from materialised
+    softmaxes (scipy), and is non-negative."""
+    d = 64
+    q1, k1, q2, k2 = make(1, 2, 2, 17, 40, d, 21)
+    fwd12, _, _ = oracle.fwd(q1, k1, q2, k2)
+    fwd21, _, _ = oracle.fwd(q2, k2, q1, k1)
+    s1 = np.einsum("bhid,bhjd->bhij", q1, k1) / 8.0
+    s2 = np.einsum("bhid,bhjd->bhij", q2, k2) / 8.0
+    lp1 = s1 - sp.logsumexp(s1, axis=-1, keepdims=True)
+    lp2 = s2 - sp.logsumexp(s2, axis=-1, keepdims=True)
+    rev = (np.exp(lp2) * (lp2 - lp1)).sum(-1)
+    sym = ((np.exp(lp1) - np.exp(lp2)) * (lp1 - lp2)).sum(-1)
+    np.testing.assert_allclose(fwd21, rev, rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(fwd12 + fwd21, sym, rtol=1e-10, atol=1e-13)
+    assert sym.min() >= -1e-12
+    assert np.abs(fwd12 - fwd21).max() > 1e-4          # the two directions differ
+
+
 def test_causal_row_zero():
     d = 64
     q1, k1, q2, k2 = make(1, 3, 3, 9, 9, d, 10)
