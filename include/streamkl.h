@@ -104,9 +104,11 @@ int streamkl_fwd_splits(int B, int Hq, int NQ, int NK);
 size_t streamkl_fwd_splitk_workspace_bytes(int B, int Hq, int NQ, int NK, int splits);
 
 /*
- * Bytes of fp32 workspace streamkl_bwd needs for these sizes: B*Hkv*ceil(NK/128)*128*d*4
- * (the dK accumulator, whole 128-row key tiles).  Returns 0 for sizes outside the supported
- * range.
+ * Bytes of fp32 workspace streamkl_bwd needs for these sizes: the dK accumulator,
+ * B*Hkv*ceil(NK/128)*128*d*4 (whole 128-row key tiles), plus, when streamkl_bwd splits each
+ * query tile's keys into ranges (its B*Hq*ceil(NQ/128) query tiles alone would leave SMs
+ * idle and there are at least two key tiles), the dQ partial sums
+ * B*Hq*ceil(NQ/128)*128*d*4.  Returns 0 for sizes outside the supported range.
  */
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d);
 
@@ -121,6 +123,12 @@ size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int 
  *   dQ_t = scale * dS_t K_t,  dK_t = scale * dS_t^T Q_t summed over the query heads that
  *   share the KV head.  The fixed distribution gets no gradient; with k1 == k2 the
  *   returned dk is the gradient through the free distribution only.
+ * One CTA owns a 128-row query tile and visits every key tile its rows see, once ("Fusão de
+ * Kernel").  When those CTAs alone would leave SMs idle (few query rows, long keys), each
+ * tile's keys are split into ranges handled by separate CTAs and dQ is summed through the
+ * workspace too; the choice is the library's and is reflected in
+ * streamkl_bwd_workspace_bytes.  Launches: a workspace memset, the backward kernel, one
+ * convert kernel for dK (and one for dQ when the keys are split).
  *
  *   kl, lse1, lse2 : the forward's outputs for the same inputs (read only).
  *   dkl            : fp32 [B,Hq,NQ] upstream gradient (read only).
