@@ -29,6 +29,10 @@
 // MMAs of visit n still read theirs, so the tensor core is handed work without waiting for
 // the write.
 //
+// When the query tiles alone would leave SMs idle, the library splits each tile's key tiles
+// into ranges (one CTA each); dQ is then added into a second tile-blocked fp32 workspace
+// instead of being written once, and converted like dK.
+//
 // The workspace is private to the library and tile-blocked: one contiguous 128 x d block
 // per (batch, KV head, key tile), laid out [lane quarter][32-column chunk][4-column group]
 // [lane][4], the order in which the flush warps hold it; the convert kernel turns it into

@@ -3,8 +3,8 @@
 // One CTA owns 256 query rows of one (batch, query head): two 128-row tiles t = 0, 1.
 // Key tiles of 128 keys stream through a ring of shared-memory slots filled by TMA.  For
 // every key tile the tensor core computes S1 = Q1 K1^T and S2 = Q2 K2^T for both query
-// tiles into TMEM (fp32, lane = query row, column = key), and one 128-thread warpgroup per
-// query tile (one thread per row) folds the tile into the row's five running scalars
+// tiles into TMEM (fp32, lane = query row, column = key), and two 128-thread statistics
+// warpgroups (one thread per row) fold it into the rows' five running scalars
 //   m1, l1, m2, l2, acc
 // (StreamKL technical summary, gist.science, Portuguese, "1. Formulação Online (Passagem
 // Forward)"), rescaling l1, acc and l2 by 2^(m_old - m_new) whenever a maximum grows (the
@@ -13,10 +13,13 @@
 // tiles past the diagonal are never loaded or multiplied.
 //
 // Roles (384 threads):  warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
-// warps 2-3 idle, warps 4-7 = statistics warpgroup of tile 0, warps 8-11 = tile 1 (when the
-// block has one query tile, the two warpgroups instead take alternate key tiles of it).
-// Warp w may touch TMEM lanes 32*(w%4) .. 32*(w%4)+31, so each statistics warp owns the
-// 32 rows that live in its lane quarter.
+// warps 2-3 idle, warps 4-7 and 8-11 = statistics warpgroups g = 0, 1.  With two query tiles
+// warpgroup g folds key columns [64g, 64g + 64) of both tiles (one state per row and tile);
+// with one query tile the two warpgroups take alternate key tiles of it, each in its own
+// TMEM half; with at most 32 query rows the rows sit in all four lane quarters and each warp
+// folds one 32-column chunk.  The partial states of a row are combined in the CTA at the
+// end.  Warp w may touch TMEM lanes 32*(w%4) .. 32*(w%4)+31, so each statistics warp owns
+// the 32 rows that live in its lane quarter.
 //
 // Scores are kept in base-2 units: u = s_raw * scale * log2(e), where s_raw = <q, k>.
 //
