@@ -395,36 +395,62 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 if (!SHARED_K) mma_commit(BAR(C::K_EMPTY + slot_of(n, 0)));
                 return true;
             };
-            bool ok = mbar_wait(BAR(C::Q_FULL), 0, abort_flag);
-            if (ok && N > 0) ok = issue_S(0);
-            for (int n = 0; n < N && ok; ++n) {
-                if (n + 1 < N) {
-                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
-                    tc_fence_after();
-                    if (!issue_S(n + 1)) break;
-                }
-                const uint32_t ds = sb + C::kDS + (n & 1) * C::kDSBuf;
+            // dQ of visit m, once its dS tile is written (and the flush has read dK of m-1)
+            auto issue_dq = [&](int m) -> bool {
+                const uint32_t ds = sb + C::kDS + (m & 1) * C::kDSBuf;
                 const uint64_t ddsk = sw128_desc(ds, 16, 1024);         // dS, K-major (A of dQ)
-                const uint64_t ddsm = sw128_desc(ds, C::kBox, 1024);    // dS^T, MN-major (A of dK)
-                const uint64_t dkfm = sw128_desc(sb + C::kRing + slot_of(n, kJFree) * C::kTile,
+                const uint64_t dkfm = sw128_desc(sb + C::kRing + slot_of(m, kJFree) * C::kTile,
                                                  C::kBox, 1024);        // K_free, MN-major
-                if (!mbar_wait(BAR(C::DS_FULL + (n & 1)), (n >> 1) & 1, abort_flag)) break;
+                if (!mbar_wait(BAR(C::DS_FULL + (m & 1)), (m >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                // dQ += dS K_free, accumulated over every visit; it does not wait for the flush
+                // dQ += dS K_free, accumulated over every visit
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
                     mma_bf16_ss(tmem + C::kColDQ, dadd(ddsk, (k >> 2) * C::kBox + (k & 3) * 32),
-                                dadd(dkfm, k * 2048), idQ, (n > 0 || k > 0));
+                                dadd(dkfm, k * 2048), idQ, (m > 0 || k > 0));
                 }
-                mma_commit(BAR(C::K_EMPTY + slot_of(n, kJFree)));
-                // dK partial of this key tile: dS^T Q_free (fresh every visit)
+                mma_commit(BAR(C::K_EMPTY + slot_of(m, kJFree)));
+                return true;
+            };
+            // dK partial of visit m: dS^T Q_free (fresh every visit); frees its dS tile
+            auto issue_dk = [&](int m) {
+                const uint64_t ddsm = sw128_desc(sb + C::kDS + (m & 1) * C::kDSBuf, C::kBox, 1024);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
                     mma_bf16_ss(tmem + C::kColDK, dadd(ddsm, k * 2048), dadd(dqfm, k * 2048), idK,
                                 k > 0);
                 }
                 mma_commit(BAR(C::DK_FULL));
-                mma_commit(BAR(C::DS_FREE + (n & 1)));
+                mma_commit(BAR(C::DS_FREE + (m & 1)));
+            };
+            bool ok = mbar_wait(BAR(C::Q_FULL), 0, abort_flag);
+            if (ok && N > 0) ok = issue_S(0);
+            if constexpr (D == 64) {
+            // Issue order dQ(n-1), S(n+1), dK(n-1): the tensor core executes in issue order, so
+            // S(n+1) -- which the compute warps wait for -- queues behind 8 dQ MMAs instead of
+            // 16 dQ and dK MMAs.  dQ(n-1) still frees visit n-1's key slot before S(n+1); the
+            // two dS tiles cover the later dK.  Measured faster at d = 64 (GQA, mode 1: 6.83 ->
+            // 6.4 ms), slower at d = 128 (headline 4.33 -> 4.8 ms), so d = 128 keeps the order
+            // S(n+1), dQ(n), dK(n).
+            for (int n = 0; n <= N && ok; ++n) {
+                if (n >= 1 && !issue_dq(n - 1)) break;
+                if (n + 1 < N) {
+                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+                    tc_fence_after();
+                    if (!issue_S(n + 1)) break;
+                }
+                if (n >= 1) issue_dk(n - 1);
+            }
+            } else {
+            for (int n = 0; n < N && ok; ++n) {
+                if (n + 1 < N) {
+                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+                    tc_fence_after();
+                    if (!issue_S(n + 1)) break;
+                }
+                if (!issue_dq(n)) break;
+                issue_dk(n);
+            }
             }
             mma_commit(BAR(C::DQ_DONE));
             mma_commit(BAR(C::DONE));
