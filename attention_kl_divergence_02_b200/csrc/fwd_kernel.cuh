@@ -81,7 +81,8 @@ struct FwdCfg {
 // two pipes share the exponentials of a chunk.
 // Default: a quarter of each (pairs 1, 5, 9, 13 of S1 and 3, 7, 11, 15 of S2, spread so
 // the polynomial work interleaves with the exponential unit's); chosen by timing the
-// headline forward (2.75 ms with none, 2.61 ms with this split, slower with more).
+// headline forward (2.75 ms with none, 2.61 ms with this split, slower with more; at d = 64
+// a third or a half on the FMA pipe is slower too: 5.05 -> 5.23 / 5.47 ms on B4 Hq32 NK32768).
 #ifndef SKL_FWD_EMU1
 #define SKL_FWD_EMU1 0x2222u
 #endif
