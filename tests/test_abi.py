@@ -170,3 +170,41 @@ def test_header_is_plain_c():
                     'int main(void){return vfn != streamkl_version;}\n')
         subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I",
                                os.path.join(ROOT, "include"), src, "-o", os.path.join(td, "t.o")])
+
+
+def test_plain_c_program_links_and_calls_the_library(lib):
+    """A C99 program (no CUDA or torch headers) links libstreamkl.so and calls the host-only
+    entry points: version, status strings, workspace sizes, the split choice, and argument
+    rejection before any device work."""
+    import subprocess
+    import tempfile
+    libdir = os.path.dirname(build.LIB)
+    src = r'''
+#include <stdio.h>
+#include <string.h>
+#include "streamkl.h"
+int main(void) {
+    if (streamkl_version() < 100) return 1;
+    if (strcmp(streamkl_status_string(STREAMKL_OK), "ok") != 0) return 2;
+    if (streamkl_bwd_workspace_bytes(1, 32, 32, 16384, 16384, 128) != (size_t)32 * 16384 * 128 * 4) return 3;
+    if (streamkl_fwd_splits(1, 32, 16384, 16384) != 1) return 4;
+    if (streamkl_fwd_splitk_workspace_bytes(1, 1, 1, 5000, 7) != (size_t)7 * 5 * 4) return 5;
+    /* null pointers and bad shapes are refused on the host */
+    if (streamkl_fwd(NULL, NULL, NULL, NULL, 1, 1, 1, 8, 8, 64, 0.125f, 0, NULL, NULL, NULL, NULL)
+        != STREAMKL_ERR_INVALID_ARG) return 6;
+    if (streamkl_bwd(3, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 8, 8, 64, 0.125f, 0,
+                     NULL, NULL, NULL, 0, NULL) != STREAMKL_ERR_INVALID_ARG) return 7;
+    printf("ok\n");
+    return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "t.c")
+        exe = os.path.join(td, "t")
+        with open(c, "w") as f:
+            f.write(src)
+        subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), c,
+                               "-L", libdir, "-lstreamkl", "-Wl,-rpath," + libdir, "-o", exe])
+        out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+        assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+        assert out.stdout.strip() == "ok"
