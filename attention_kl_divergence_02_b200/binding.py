@@ -198,6 +198,23 @@ def _check_inputs(q1, k1, q2, k2):
         raise ValueError("q1/q2 must be [B,Hq,NQ,d], k1/k2 [B,Hkv,NK,d]")
 
 
+def _check_tensor(name, t, shape, dtype, device):
+    """Refuses a tensor the kernels would read or write out of bounds or misinterpret."""
+    if t is None:
+        raise ValueError("%s is required" % name)
+    if t.dtype != dtype or t.device != device or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must be a contiguous %s tensor of shape %s on %s (got %s %s on %s)"
+                         % (name, dtype, tuple(shape), device, t.dtype, tuple(t.shape), t.device))
+
+
+def _check_workspace(workspace, nbytes, device):
+    if workspace.device != device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on %s" % device)
+    have = workspace.numel() * workspace.element_size()
+    if have < nbytes:
+        raise ValueError("workspace holds %d bytes, %d needed" % (have, nbytes))
+
+
 def fwd(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
     """Returns (kl, lse1, lse2), fp32 [B,Hq,NQ].  Pass k2 = k1 (same tensor) for shared keys."""
     import torch
@@ -206,6 +223,8 @@ def fwd(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if out is None:
         out = tuple(torch.empty((B, Hq, NQ), dtype=torch.float32, device=q1.device) for _ in range(3))
+    for name, o in zip(("kl", "lse1", "lse2"), out):
+        _check_tensor(name, o, (B, Hq, NQ), torch.float32, q1.device)
     rc = streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, *out, stream=stream)
     if rc != OK:
         raise StreamKLError(rc, "streamkl_fwd")
@@ -222,9 +241,13 @@ def fwd_splitk(q1, k1, q2, k2, scale=None, causal=False, splits=0, out=None, wor
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if out is None:
         out = tuple(torch.empty((B, Hq, NQ), dtype=torch.float32, device=q1.device) for _ in range(3))
+    for name, o in zip(("kl", "lse1", "lse2"), out):
+        _check_tensor(name, o, (B, Hq, NQ), torch.float32, q1.device)
     need = streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits)
     if workspace is None and need > 0:
         workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q1.device)
+    if workspace is not None:
+        _check_workspace(workspace, need, q1.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = streamkl_fwd_splitk(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, *out,
                              workspace, wbytes, stream=stream)
@@ -240,11 +263,16 @@ def bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, scale=None, causal=False, out
     _check_inputs(q1, k1, q2, k2)
     B, Hq, Hkv, NQ, NK, d = _dims(q1, k1)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    for name, v in zip(("kl", "lse1", "lse2", "dkl"), (kl, lse1, lse2, dkl)):
+        _check_tensor(name, v, (B, Hq, NQ), torch.float32, q1.device)
     if out is None:
         out = (torch.empty_like(q1), torch.empty_like(k1))
+    _check_tensor("dq", out[0], q1.shape, torch.bfloat16, q1.device)
+    _check_tensor("dk", out[1], k1.shape, torch.bfloat16, q1.device)
     nbytes = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16) // 4, dtype=torch.float32, device=q1.device)
+    _check_workspace(workspace, nbytes, q1.device)
     rc = streamkl_bwd(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
                       causal, out[0], out[1], workspace, workspace.numel() * workspace.element_size(),
                       stream=stream)

@@ -197,3 +197,26 @@ def test_upstream_gradient_signs_and_zeros(case, kind, mode):
     check_grad(dk, odk, "%s %s dK mode %d" % (case, kind, mode), zero_atol)
     if kind == "zeros":
         assert np.abs(dq[..., ::3, :]).max() <= 1e-30
+
+
+def test_binding_refuses_mismatched_tensors_before_launch():
+    """The Python wrappers check every tensor the kernels would read or write (dtype, shape,
+    contiguity, device) and the workspace size before calling the library."""
+    w = inputs.custom(1, 2, 2, 128, 128, 64, False, True, seed=3)
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"])
+    with pytest.raises(ValueError):
+        binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], out=(kl, l1, torch.empty(1, 2, 64, device="cuda")))
+    with pytest.raises(ValueError):
+        binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"].half())
+    with pytest.raises(ValueError):
+        binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"],
+                    out=(torch.empty_like(t["q1"]), torch.empty(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")))
+    need = binding.streamkl_bwd_workspace_bytes(1, 2, 2, 128, 128, 64)
+    with pytest.raises(ValueError):
+        binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"],
+                    workspace=torch.empty(need // 4 - 1, device="cuda"))
+    with pytest.raises(ValueError):
+        binding.fwd_splitk(t["q1"], t["k1"], t["q2"], t["k2"], splits=2,
+                           workspace=torch.empty(1, device="cuda"))
+    assert binding.streamkl_device_status() == binding.OK
