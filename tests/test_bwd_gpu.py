@@ -216,7 +216,10 @@ def test_binding_refuses_mismatched_tensors_before_launch():
     with pytest.raises(ValueError):
         binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"],
                     workspace=torch.empty(need // 4 - 1, device="cuda"))
+    w2 = inputs.custom(1, 2, 2, 1, 1024, 64, False, True, seed=4)     # 8 key tiles: a real split
+    t2 = inputs.make(w2, device="cuda")
+    assert binding.streamkl_fwd_splitk_workspace_bytes(1, 2, 1, 1024, 2) > 4
     with pytest.raises(ValueError):
-        binding.fwd_splitk(t["q1"], t["k1"], t["q2"], t["k2"], splits=2,
+        binding.fwd_splitk(t2["q1"], t2["k1"], t2["q2"], t2["k2"], splits=2,
                            workspace=torch.empty(1, device="cuda"))
     assert binding.streamkl_device_status() == binding.OK
