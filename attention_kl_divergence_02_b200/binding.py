@@ -35,6 +35,8 @@ EXPORTS = (
     "streamkl_selftest_watchdog",
     "streamkl_last_cuda_error",
     "streamkl_version",
+    "streamkl_probe_exp2",
+    "streamkl_num_sms",
 )
 
 _lib = None
@@ -86,6 +88,10 @@ def load(path=None):
     lib.streamkl_last_cuda_error.restype = ctypes.c_char_p
     lib.streamkl_version.argtypes = []
     lib.streamkl_version.restype = i
+    lib.streamkl_probe_exp2.argtypes = [i, i, ctypes.POINTER(ctypes.c_longlong), vp]
+    lib.streamkl_probe_exp2.restype = i
+    lib.streamkl_num_sms.argtypes = []
+    lib.streamkl_num_sms.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -146,9 +152,10 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 def streamkl_bwd_noalloc(mode, q1, k1, q2, k2, kl, lse1, lse2, dkl, B, Hq, Hkv, NQ, NK, d, scale,
                          causal, dq, dk, stream=None):
     """Backward without a workspace argument, for callers that may not allocate device
-    memory: the library's fixed 32 MiB built-in buffer holds the dK accumulator.  Calls
-    that can overlap on the GPU share that buffer and race; larger problems return
-    ERR_UNSUPPORTED."""
+    memory: the library's fixed 32 MiB built-in buffer holds what streamkl_bwd keeps in its
+    workspace (the dK accumulator, plus the dQ partial sums when keys are split into ranges),
+    so sizes with streamkl_bwd_workspace_bytes(...) > 32 MiB return ERR_UNSUPPORTED.  Calls
+    that can overlap on the GPU share that buffer and race."""
     return load().streamkl_bwd_noalloc(int(mode), _ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), _ptr(kl),
                                        _ptr(lse1), _ptr(lse2), _ptr(dkl), B, Hq, Hkv, NQ, NK, d,
                                        float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
@@ -168,6 +175,17 @@ def streamkl_selftest_watchdog(starve, stream=None):
     ns = (ctypes.c_longlong * 2)()
     rc = load().streamkl_selftest_watchdog(int(starve), ns, _stream(stream))
     return rc, [ns[0], ns[1]]
+
+
+def streamkl_probe_exp2(kind, iters, stream=None):
+    """Launches the exponential-throughput probe; returns (status, exponentials evaluated)."""
+    n = ctypes.c_longlong(0)
+    rc = load().streamkl_probe_exp2(int(kind), int(iters), ctypes.byref(n), _stream(stream))
+    return rc, n.value
+
+
+def streamkl_num_sms():
+    return load().streamkl_num_sms()
 
 
 def status_string(status):
@@ -190,12 +208,23 @@ def _dims(q1, k1):
 
 
 def _check_inputs(q1, k1, q2, k2):
+    """Refuses inputs whose shapes or devices disagree: the library sizes every tensor map
+    from q1's batch and head dimension and k1's key count, so a mismatch would make a kernel
+    read past an allocation."""
     import torch
     for t in (q1, k1, q2, k2):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("inputs must be contiguous bf16 CUDA tensors")
-    if q1.shape != q2.shape or k1.shape != k2.shape or q1.dim() != 4 or k1.dim() != 4:
+    if q1.dim() != 4 or k1.dim() != 4 or q1.shape != q2.shape or k1.shape != k2.shape:
         raise ValueError("q1/q2 must be [B,Hq,NQ,d], k1/k2 [B,Hkv,NK,d]")
+    if q1.shape[0] != k1.shape[0] or q1.shape[3] != k1.shape[3]:
+        raise ValueError("q and k must share batch size and head dim (q %s, k %s)"
+                         % (tuple(q1.shape), tuple(k1.shape)))
+    if k1.shape[1] < 1 or q1.shape[1] % k1.shape[1] != 0:
+        raise ValueError("query heads (%d) must be a multiple of KV heads (%d)"
+                         % (q1.shape[1], k1.shape[1]))
+    if len({t.device for t in (q1, k1, q2, k2)}) != 1:
+        raise ValueError("q1, k1, q2, k2 must be on one device")
 
 
 def _check_tensor(name, t, shape, dtype, device):

@@ -140,35 +140,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
-// 16 consecutive fp32 TMEM columns of the thread's lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-// 8 consecutive fp32 TMEM columns of the thread's lane.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-}
-
-// tcgen05.wait::ld that also names the 16 registers the outstanding loads write, so that
-// no use of them can be scheduled above the wait.
-__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[8], uint32_t (&b)[8]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]),
-                   "+r"(a[6]), "+r"(a[7]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]),
-                   "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])
-                 :: "memory");
-}
-
 // Which of a chunk's four column pairs take their P2 exponential on the FMA pipe instead of
 // the exponential unit (mode 1 only; mode 2 has one exponential per element and leaves the
 // unit half idle).  Two of the chunk's eight exponential pairs = a quarter of the mode-1
@@ -508,14 +479,17 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             bq = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
             g = p.dkl[o];
         }
-        // fold g into the exponents when no row of the warp has g < 0 (log2 0 = -inf makes
-        // a row with g = 0 give exactly 0)
+        // fold g into the exponents when no row of the warp has g < 0
         const bool folded = !__any_sync(0xffffffffu, g < 0.f);
-        if (folded) {
+        if (folded && g > 0.f) {
             const float lg = log2f(g);
             a -= lg;
             if (mode1) bq -= lg;
         }
+        // a row with g = 0 (or past NQ) has dS = 0 exactly: it takes the masked variant with
+        // every column masked (folding log2 0 = -inf would leave 2^-126 where the FMA-pipe
+        // exponential clamps its argument)
+        const bool zero_row = !(g != 0.f);
         const int kc0 = wg * 32;
         bool ok = true;
         for (int n = 0; n < N; ++n) {
@@ -523,11 +497,15 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             const int k0 = kt * 128;
             // masked columns: keys past the diagonal of a causal diagonal tile, and
             // zero-filled keys past NK; columns k < lim of this warpgroup are valid
-            const bool need_mask = (p.causal && kt == qt) || (k0 + 128 > p.NK);
+            bool need_mask = (p.causal && kt == qt) || (k0 + 128 > p.NK);
             int lim = 32;
             if (need_mask) {
                 lim = min(lim, p.NK - k0 - kc0);
                 if (p.causal && kt == qt) lim = min(lim, r - kc0 + 1);
+            }
+            if (zero_row) {
+                need_mask = true;
+                lim = 0;
             }
             if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
                 ok = false;

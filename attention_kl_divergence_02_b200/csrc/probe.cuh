@@ -1,0 +1,49 @@
+// probe.cuh -- throughput probe of the two exponential paths the kernels use: the
+// exponential unit (ex2.approx on the MUFU) and the FMA-pipe polynomial ex2_poly2.  The
+// StreamKL forward spends two exponentials per (row, key) pair and has no second GEMM to
+// amortise them (StreamKL technical summary, gist.science, Portuguese, "1. Formulação
+// Online"), so the rate of these two paths, not the tensor core, sets its floor; the bench
+// divides a kernel's exponential count by the rates measured here.
+//
+// Every thread runs kChains independent recurrences y <- 2^(c - y/2) (values stay in
+// (0.5, 2], so neither path over- or underflows); each step is one exponential and one FMA
+// that forms its argument.  Nothing else is in the loop, and the sum of the chains goes to a
+// store that the host never enables, so the compiler must keep every exponential.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace skl {
+
+constexpr int kProbeChains = 8;
+constexpr int kProbeThreads = 256;
+
+template <int KIND>   // 0: MUFU ex2.approx; 1: ex2_poly2 on the FMA/ALU pipes
+__global__ void __launch_bounds__(kProbeThreads)
+streamkl_probe_exp2_kernel(int iters, int write, float* sink) {
+    float y[kProbeChains];
+#pragma unroll
+    for (int k = 0; k < kProbeChains; ++k) y[k] = 1.0f + 0.01f * (float)((threadIdx.x + k) & 7);
+#pragma unroll 1
+    for (int i = 0; i < iters; ++i) {
+        if (KIND == 0) {
+#pragma unroll
+            for (int k = 0; k < kProbeChains; ++k) y[k] = ex2(fmaf(y[k], -0.5f, 0.125f));
+        } else {
+#pragma unroll
+            for (int k = 0; k < kProbeChains; k += 2) {
+                const float2 u = __ffma2_rn(make_float2(y[k], y[k + 1]), make_float2(-0.5f, -0.5f),
+                                            make_float2(0.125f, 0.125f));
+                const float2 e = ex2_poly2(u);
+                y[k] = e.x;
+                y[k + 1] = e.y;
+            }
+        }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < kProbeChains; ++k) s += y[k];
+    if (write) sink[blockIdx.x * kProbeThreads + threadIdx.x] = s;
+}
+
+}  // namespace skl

@@ -16,6 +16,7 @@
 #include "fwd_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "watchdog.cuh"
+#include "probe.cuh"
 
 namespace {
 
@@ -68,6 +69,31 @@ int make_map(CUtensorMap* map, const void* base, long long planes, long long row
     return STREAMKL_OK;
 }
 
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultSMs = 148;   // B200; used only when no device can be queried
+
+// SM count of the current device, looked up once per device ordinal (it cannot change while
+// the process runs).  The split heuristics size their grids in waves of one CTA per SM.
+int num_sms() {
+    static std::mutex mu;
+    static int cache[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();   // no device here (host-only queries): clear and use the default
+        return kDefaultSMs;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            return kDefaultSMs;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal) {
@@ -107,7 +133,8 @@ int launch_convert(const float* ws, uint16_t* out, int planes, int rows, int nti
                    cudaStream_t st, const char* what) {
     const size_t threads = (size_t)planes * ntiles * 128 * (D / 32);
     size_t blocks = (threads + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    const size_t cap = (size_t)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
     skl::streamkl_tile_convert_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(ws, out, planes, rows, ntiles,
                                                                           scale);
     cudaError_t e = cudaGetLastError();
@@ -189,11 +216,28 @@ int streamkl_selftest_watchdog(int starve, long long* waited_ns, void* stream) {
     return status;
 }
 
+
+int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream) {
+    if ((kind != 0 && kind != 1) || iters < 1) return STREAMKL_ERR_INVALID_ARG;
+    const int grid = 4 * num_sms();
+    const long long n = (long long)grid * skl::kProbeThreads * skl::kProbeChains * iters;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == 0)
+        skl::streamkl_probe_exp2_kernel<0><<<grid, skl::kProbeThreads, 0, st>>>(iters, 0, nullptr);
+    else
+        skl::streamkl_probe_exp2_kernel<1><<<grid, skl::kProbeThreads, 0, st>>>(iters, 0, nullptr);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "exp2 probe launch");
+    if (n_exp) *n_exp = n;
+    return STREAMKL_OK;
+}
+
+int streamkl_num_sms(void) { return num_sms(); }
+
 }  // extern "C"
 
 namespace {
 
-constexpr int kNumSMs = 148;
 
 // Key tiles per range for `splits` ranges, and the number of non-empty ranges that gives.
 void split_ranges(int NK, int splits, int* kps, int* used) {
@@ -238,7 +282,7 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
     }
     if (rc || p.splits == 1) return rc;
     const long long R = (long long)B * Hq * NQ;
-    const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * kNumSMs);
+    const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * num_sms());
     skl::streamkl_splitk_merge_kernel<<<mgrid, 256, 0, st>>>(part, p.splits, R, scale, kl, lse1, lse2);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
@@ -266,7 +310,8 @@ int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
     if (B < 1 || Hq < 1 || NQ < 1 || NK < 1) return 1;
     const long long blocks = (long long)B * Hq * ((NQ + 255) / 256);
     const int nkt = (NK + 127) / 128;
-    if (blocks >= kNumSMs || nkt < 2) return 1;
+    const int sms = num_sms();
+    if (blocks >= sms || nkt < 2) return 1;
     // time model: waves of one CTA per SM, each CTA ~ its key tiles + 8 tiles of fixed cost
     // (query load, pipeline fill and drain, partial store; 8 measured on B4 H32 NQ1 NK32768,
     // where 128 blocks already fill the GPU and splitting lost 6 %); the fewest ranges within
@@ -278,7 +323,7 @@ int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
         int kps, used;
         split_ranges(NK, s, &kps, &used);
         const long long ctas = blocks * used;
-        const double waves = (double)((ctas + kNumSMs - 1) / kNumSMs);
+        const double waves = (double)((ctas + sms - 1) / sms);
         cost[s] = waves * (kps + 8);
         if (cost[s] < best) best = cost[s];
     }
@@ -329,13 +374,14 @@ namespace {
 int bwd_splits(int B, int Hq, int NQ, int NK) {
     const long long ctas = (long long)B * Hq * ((NQ + 127) / 128);
     const int nkt = (NK + 127) / 128;
-    if (ctas >= kNumSMs || nkt < 2) return 1;
+    const int sms = num_sms();
+    if (ctas >= sms || nkt < 2) return 1;
     double cost[33] = {0};
     double best = 1e300;
     for (int s = 1; s <= std::min(nkt, 32); ++s) {
         int kps, used;
         split_ranges(NK, s, &kps, &used);
-        const double waves = (double)((ctas * used + kNumSMs - 1) / kNumSMs);
+        const double waves = (double)((ctas * used + sms - 1) / sms);
         cost[s] = waves * (kps + 6);
         best = std::min(best, cost[s]);
     }
@@ -419,19 +465,51 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
 
 // ------------------------------------------------------------------ no-allocation backward
 // The scratch buffer behind streamkl_bwd_noalloc: a fixed-size static device array, so the
-// entry point never allocates.  Host code must not pass `g_noalloc_dq_scratch` itself to a
-// kernel (on the host that name is only a stand-in for the symbol); it passes the device
-// address that cudaGetSymbolAddress returns, looked up once per device.
-static __device__ __align__(256) float g_noalloc_dq_scratch[STREAMKL_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+// entry point never allocates.  It holds whatever streamkl_bwd would keep in its workspace:
+// the fp32 dK accumulator, plus the fp32 dQ partial sums when the key-range split is chosen.
+// Host code must not pass `g_noalloc_scratch` itself to a kernel (on the host that name is
+// only a stand-in for the symbol); it passes the device address that cudaGetSymbolAddress
+// returns, looked up with the device current.
+static __device__ __align__(256) float g_noalloc_scratch[STREAMKL_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 float* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (first call per device does
-// the lookup with that device current).  Returns nullptr and sets the error text on failure.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (ids are never reused, unlike
+// context handles), or 0 when there is none yet or the driver cannot say.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+        looked = true;
+    }
+    if (!get_cur || !get_id) return 0;
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_cur(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch array on the current device.  The lookup is done the first
+// time a device is used, with that device current, and again whenever that device's context
+// has changed since (a cudaDeviceReset destroys the context and the module with it, so the
+// old address is no longer valid).  Returns nullptr and sets the error text on failure.
 float* noalloc_scratch() {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -445,14 +523,16 @@ float* noalloc_scratch() {
         return nullptr;
     }
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_dq_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr) {
             cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
             return nullptr;
         }
         g_noalloc_ptr[dev] = static_cast<float*>(p);
+        g_noalloc_ctx[dev] = current_context_id();   // the lookup made the context current
     }
     return g_noalloc_ptr[dev];
 }

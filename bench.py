@@ -79,6 +79,95 @@ def job_tflops(world, flops_per_rank_step, ms_per_step):
     return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
+# ------------------------------------------------------------------ roofline bookkeeping
+# Share of the forward's exponentials that the kernel evaluates with the FMA-pipe polynomial
+# instead of the exponential unit: 4 of the 16 column pairs of every 32-column chunk, for S1
+# and for S2 (the kEmu1 / kEmu2 masks of the forward kernel).
+FWD_POLY_SHARE = 0.25
+
+
+def choose_peak(peaks, peak_src, timed_s, clk):
+    """The bf16 denominator of a tensor-bound call: the burst figure when the timed region is
+    short (under a second) and the sampled SM clock stayed at its maximum -- the conditions
+    the burst GEMM was measured in -- else the sustained figure (a seconds-long loop under
+    the power cap).  Returns (peak, label, reason)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    med, mx = (clk or {}).get("sm_mhz"), (clk or {}).get("sm_max_mhz")
+    at_max = med is not None and mx is not None and med >= 0.97 * mx
+    if timed_s < 1.0 and at_max:
+        return burst, "%s bf16_tflops (burst)" % peak_src, (
+            "timed region %.2f s < 1 s and median SM clock %.0f MHz at its maximum %.0f"
+            % (timed_s, med, mx))
+    why = []
+    if timed_s >= 1.0:
+        why.append("timed region %.2f s >= 1 s" % timed_s)
+    if not at_max:
+        why.append("median SM clock %s MHz below its maximum %s" % (med, mx))
+    return sus, "%s bf16_tflops_sustained" % peak_src, "; ".join(why)
+
+
+def measure_exp_rates(binding, stream, gpu_index, target_ms=120.0):
+    """Throughput of the two exponential paths (library probe: MUFU ex2.approx, and the
+    FMA-pipe polynomial), each timed alone with CUDA events over ~target_ms, best of three,
+    with the SM clock sampled meanwhile.  Returns exponentials per SM per clock for each
+    path, with the clock and the raw rate they come from."""
+    import torch
+    sms = binding.streamkl_num_sms()
+    out = {}
+    clocks = ClockSampler(gpu_index, tag="exp")
+    clocks.start()
+    time.sleep(0.3)
+    for kind, name in ((0, "mufu_ex2"), (1, "fma_poly")):
+        def run(iters):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rc, n = binding.streamkl_probe_exp2(kind, iters, stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if rc != binding.OK:
+                raise RuntimeError("exp2 probe: %s" % binding.status_string(rc))
+            return a.elapsed_time(b), n
+        run(64)
+        ms, _ = run(2000)
+        iters = max(2000, int(2000 * target_ms / max(ms, 1e-3)))
+        best = None
+        for _ in range(3):
+            ms, n = run(iters)
+            rate = n / (ms * 1e-3)
+            best = rate if best is None or rate > best else best
+        out[name] = {"exps_per_s": best, "iters": iters}
+    clk = clocks.stop()
+    mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+    for v in out.values():
+        v["per_sm_per_clk"] = v["exps_per_s"] / (sms * mhz * 1e6)
+        v["sm_mhz"] = mhz
+    out["sms"] = sms
+    out["clocks"] = clk
+    return out
+
+
+def exp_roofline(w, fwd_ms, rates, step_mhz):
+    """The forward's exponential-unit roof: 2 exponentials per unmasked pair (causal pairs
+    halved, as for the FLOPs), of which (1 - FWD_POLY_SHARE) run on the exponential unit; at
+    the measured MUFU rate per SM per clock and the step's median SM clock, the shortest
+    time that unit allows, divided by the forward's measured time."""
+    exps = 2.0 * w.pairs()
+    mufu = rates["mufu_ex2"]["per_sm_per_clk"] * rates["sms"] * step_mhz * 1e6   # exps / s
+    poly = rates["fma_poly"]["per_sm_per_clk"] * rates["sms"] * step_mhz * 1e6
+    t_mufu = (1.0 - FWD_POLY_SHARE) * exps / mufu
+    return {"bound": "exp", "unit": "exp2/s", "exps_per_call": exps,
+            "achieved": exps / (fwd_ms * 1e-3), "mufu_share": 1.0 - FWD_POLY_SHARE,
+            "mufu_peak": mufu, "poly_peak": poly,
+            "mufu_per_sm_per_clk": rates["mufu_ex2"]["per_sm_per_clk"],
+            "poly_per_sm_per_clk": rates["fma_poly"]["per_sm_per_clk"],
+            "frac": t_mufu * 1e3 / fwd_ms,
+            "t_mufu_ms": t_mufu * 1e3, "t_all_on_mufu_ms": exps / mufu * 1e3,
+            "note": "frac = time the exponential unit needs for its share of the forward's "
+                    "exponentials at the measured rate and the step's median clock / forward time"}
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -87,10 +176,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, tag="step"):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(tempfile.gettempdir(), "streamkl_clocks_rank%d.csv" % gpu_index)
+        self.path = os.path.join(tempfile.gettempdir(),
+                                 "streamkl_clocks_%s_rank%d.csv" % (tag, gpu_index))
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -397,16 +487,20 @@ def run_gpu(args):
                        "reads its result (KL, LSE1, LSE2) back"}
 
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # the calls are timed inside a step repeated back to back under the power cap: the
-    # roofline takes the sustained GEMM figure, the burst one is reported beside it
-    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_label, peak_reason = choose_peak(peaks, peak_src, total_ms * 1e-3, clk)
     calls = {"fwd": (f_ms, w.fwd_flops()), "bwd_mode1": (b1_ms, w.bwd_flops()),
              "bwd_mode2": (b2_ms, w.bwd_flops())}
+    tflops = {k: fl / (ms * 1e-3) / 1e12 for k, (ms, fl) in calls.items()}
     dom = max(calls, key=lambda k: calls[k][0])
-    dom_ms, dom_flops = calls[dom]
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    achieved = tflops[dom]
     traffic = load_traffic(dom)
+    exp_roof = None
+    if not args.skip_exp:
+        rates = measure_exp_rates(binding, stream, local)
+        step_mhz = clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"]
+        exp_roof = exp_roofline(w, f_ms, rates, step_mhz)
+        exp_roof["probe_clocks"] = rates["clocks"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -417,25 +511,29 @@ def run_gpu(args):
                    "global_batch": world * B, "seq_len": NQ, "heads": Hq, "head_dim": d,
                    "parallelism": "dp%d (independent batch per GPU, no collective)" % world,
                    "l2": "inputs (3 x 128 MiB bf16) larger than the 126 MB L2; no flush"},
-        "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / (f_ms * 1e-3) / 1e12,
-        "bwd_mode1_ms": b1_ms, "bwd_mode1_tflops": w.bwd_flops() / (b1_ms * 1e-3) / 1e12,
-        "bwd_mode2_ms": b2_ms, "bwd_mode2_tflops": w.bwd_flops() / (b2_ms * 1e-3) / 1e12,
-        "pct_of_peak": {"fwd": 100 * w.fwd_flops() / (f_ms * 1e-3) / 1e12 / peak,
-                        "bwd_mode1": 100 * w.bwd_flops() / (b1_ms * 1e-3) / 1e12 / peak,
-                        "bwd_mode2": 100 * w.bwd_flops() / (b2_ms * 1e-3) / 1e12 / peak,
-                        "step": 100 * value / world / peak,
+        "fwd_ms": f_ms, "fwd_tflops": tflops["fwd"],
+        "bwd_mode1_ms": b1_ms, "bwd_mode1_tflops": tflops["bwd_mode1"],
+        "bwd_mode2_ms": b2_ms, "bwd_mode2_tflops": tflops["bwd_mode2"],
+        "pct_of_peak": {"fwd": 100 * tflops["fwd"] / burst,
+                        "bwd_mode1": 100 * tflops["bwd_mode1"] / burst,
+                        "bwd_mode2": 100 * tflops["bwd_mode2"] / burst,
+                        "step": 100 * value / world / burst,
                         "basis": "%s bf16 %.1f TFLOP/s (burst); nominal dense %.0f gives fwd %.1f%%"
-                                 % (peak_src, peak, NOMINAL_BF16_TFLOPS,
-                                    100 * w.fwd_flops() / (f_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS)},
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sus,
-                     "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
-                     "peak_source": "%s bf16_tflops_sustained (timed inside a step repeated "
-                                    "back to back)" % peak_src,
-                     "peak_burst": peak, "frac_of_burst": achieved / peak,
+                                 % (peak_src, burst, NOMINAL_BF16_TFLOPS,
+                                    100 * tflops["fwd"] / NOMINAL_BF16_TFLOPS)},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "fwd_frac": tflops["fwd"] / peak, "bwd_mode1_frac": tflops["bwd_mode1"] / peak,
+                     "bwd_mode2_frac": tflops["bwd_mode2"] / peak,
+                     "peak_source": peak_label, "peak_rule": peak_reason,
+                     "peak_burst": burst, "frac_of_burst": achieved / burst,
+                     "peak_sustained": float(peaks.get("bf16_tflops_sustained",
+                                                       FALLBACK_PEAKS["bf16_tflops_sustained"])),
                      "note": "achieved = algorithmic FLOPs per call / CUDA-event duration of the "
                              "call on its stream%s" % (
-                                 "; the backward call also runs the dQ-workspace memset and the "
+                                 "; the backward call also runs the workspace memset and the "
                                  "dK convert kernel" if dom.startswith("bwd") else "")},
+        "exp_roofline": exp_roof,
         "clocks": clk,
         "gpu_launches": 5 * args.steps,
         "e2e": e2e,
@@ -619,6 +717,113 @@ def run_chunk(args):
     return 0
 
 
+CONFIG_RUNS = {
+    # name: (workload, causal override or None)
+    "b2h8n4k": ("b2h8n4k", True),
+    "b2h8n4k_noncausal": ("b2h8n4k", False),
+    "long64k": ("long64k", None),
+    "gqa": ("gqa", None),
+    "headline": ("headline", None),
+}
+
+
+def run_config(args):
+    """One JSON line for one workload: forward and both backward settings, ms and TFLOP/s per
+    call, % of the bf16 peak, the forward's exponential-unit fraction and the fp64 oracle
+    timed on a sample of the same workload beside them.  Not the driver's step line: the
+    per-workload breakdown behind it."""
+    import torch
+
+    from attention_kl_divergence_02_b200 import binding, inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--config measures one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    binding.load()
+    wname, causal = CONFIG_RUNS[args.config]
+    w = inputs.WORKLOADS[wname]
+    if causal is not None:
+        w = inputs.variant(w, causal=causal)
+    t = inputs.make(w, device=dev)
+    B, Hq, NQ, d = w.B, w.Hq, w.NQ, w.d
+    stream = torch.cuda.current_stream()
+    kl, l1, l2 = (torch.empty((B, Hq, NQ), device=dev) for _ in range(3))
+    g = (torch.empty_like(t["q1"]), torch.empty_like(t["k1"]))
+    ws = torch.empty(max(16, binding.streamkl_bwd_workspace_bytes(B, Hq, w.Hkv, NQ, w.NK, d)) // 4,
+                     device=dev)
+
+    def fwd():
+        binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal,
+                    out=(kl, l1, l2), stream=stream)
+
+    def bwd(mode):
+        binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], scale=w.scale,
+                    causal=w.causal, out=g, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        fwd(); bwd(1); bwd(2)
+    torch.cuda.synchronize()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        fwd()
+        ev[k][1].record(stream)
+        bwd(1)
+        ev[k][2].record(stream)
+        bwd(2)
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = binding.streamkl_device_status()
+    if st != binding.OK:
+        raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
+    ms = [sum(e[i].elapsed_time(e[i + 1]) for e in ev) / args.steps for i in range(3)]
+    total_s = sum(ms) * args.steps * 1e-3
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_label, peak_reason = choose_peak(peaks, peak_src, total_s, clk)
+    fl = [w.fwd_flops(), w.bwd_flops(), w.bwd_flops()]
+    tf = [f / (m * 1e-3) / 1e12 for f, m in zip(fl, ms)]
+    rates = measure_exp_rates(binding, stream, local)
+    exp_roof = exp_roofline(w, ms[0], rates, clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"])
+    line = {
+        "metric": "per-workload fwd/bwd ms and TFLOP/s; % of B200 dense bf16 peak",
+        "value": sum(fl) / (sum(ms) * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(ms),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "%s: %s%s" % (wname, w.note,
+                                             "" if causal is None else (" [causal]" if causal else " [non-causal]")),
+                   "B": B, "Hq": Hq, "Hkv": w.Hkv, "NQ": NQ, "NK": w.NK, "d": d,
+                   "causal": w.causal, "shared_k": w.shared_k},
+        "fwd_ms": ms[0], "fwd_tflops": tf[0],
+        "bwd_mode1_ms": ms[1], "bwd_mode1_tflops": tf[1],
+        "bwd_mode2_ms": ms[2], "bwd_mode2_tflops": tf[2],
+        "pct_of_burst_peak": {"fwd": 100 * tf[0] / burst, "bwd_mode1": 100 * tf[1] / burst,
+                              "bwd_mode2": 100 * tf[2] / burst,
+                              "basis": "%s bf16 %.1f TFLOP/s (burst)" % (peak_src, burst)},
+        "roofline": {"bound": "tensor", "peak": peak, "unit": "TFLOP/s", "peak_source": peak_label,
+                     "peak_rule": peak_reason, "fwd_frac": tf[0] / peak,
+                     "bwd_mode1_frac": tf[1] / peak, "bwd_mode2_frac": tf[2] / peak},
+        "exp_roofline": exp_roof,
+        "clocks": clk,
+        "gpu_launches": 5 * args.steps,
+    }
+    if not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, target_s=10.0)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary
     (profiles/dram_traffic.txt, lines "<call> <bytes>"), or None."""
@@ -642,10 +847,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU-oracle baseline leg")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer leg")
+    ap.add_argument("--skip-exp", action="store_true",
+                    help="omit the exponential-throughput probe (and the forward's exp roofline)")
     ap.add_argument("--decode", action="store_true",
                     help="measure the split-K forward on the decode workload instead of the step")
     ap.add_argument("--chunk", action="store_true",
                     help="measure the key-range backward on the chunk workload instead of the step")
+    ap.add_argument("--config", choices=sorted(CONFIG_RUNS),
+                    help="measure one workload (forward + both backward settings) instead of the step")
     ap.add_argument("--heads", type=int, default=32,
                     help="query/KV heads (32 = the headline workload; fewer only for profiler captures)")
     args = ap.parse_args()
@@ -657,6 +866,8 @@ def main():
         return run_decode(args)
     if args.chunk:
         return run_chunk(args)
+    if args.config:
+        return run_config(args)
     return run_gpu(args)
 
 

@@ -14,7 +14,8 @@
  *
  * Conventions shared by every entry point:
  *  - Every pointer argument is a DEVICE pointer owned by the caller; the library keeps no
- *    reference after the call returns and allocates no device memory.
+ *    reference after the call returns and allocates no device memory (its only device
+ *    memory of its own is the static buffer of streamkl_bwd_noalloc and a status word).
  *  - Tensors are dense and row-major with the head dimension innermost:
  *      Q1, Q2, dQ : bf16 [B, Hq, NQ, d]        K1, K2, dK : bf16 [B, Hkv, NK, d]
  *      kl, lse1, lse2, dkl : fp32 [B, Hq, NQ]
@@ -108,7 +109,9 @@ size_t streamkl_fwd_splitk_workspace_bytes(int B, int Hq, int NQ, int NK, int sp
  * B*Hkv*ceil(NK/128)*128*d*4 (whole 128-row key tiles), plus, when streamkl_bwd splits each
  * query tile's keys into ranges (its B*Hq*ceil(NQ/128) query tiles alone would leave SMs
  * idle and there are at least two key tiles), the dQ partial sums
- * B*Hq*ceil(NQ/128)*128*d*4.  Returns 0 for sizes outside the supported range.
+ * B*Hq*ceil(NQ/128)*128*d*4.  Returns 0 for sizes outside the supported range.  The split
+ * decision depends on the SM count of the current device (streamkl_num_sms), so query with
+ * the device current that the backward will run on.
  */
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d);
 
@@ -159,14 +162,18 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
  * device-wide synchronisation that cudaMalloc/cudaFree can cause.
  *
  * Same arguments, semantics and outputs as streamkl_bwd, minus workspace/workspace_bytes:
- * the fp32 dK accumulator lives in a fixed STREAMKL_NOALLOC_SCRATCH_BYTES (32 MiB) buffer
- * compiled into the library as a static device array.  Every GPU on which the library is
- * loaded holds that buffer until the process exits.
- *  - Sizes whose workspace (streamkl_bwd_workspace_bytes) exceeds the buffer return
+ * what streamkl_bwd keeps in its workspace -- the fp32 dK accumulator, plus the fp32 dQ
+ * partial sums when the key-range split is chosen -- lives in a fixed
+ * STREAMKL_NOALLOC_SCRATCH_BYTES (32 MiB) buffer compiled into the library as a static
+ * device array.  Every GPU on which the library is loaded holds that buffer until the
+ * process exits.
+ *  - The limit: streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d) <= 32 MiB (for example
+ *    at most 4 KV heads of 16384 keys at d = 128).  Larger sizes return
  *    STREAMKL_ERR_UNSUPPORTED and launch nothing; use streamkl_bwd for those.
- *  - The first call on each device looks up the buffer's device address (a one-time
- *    set-up done with that device current); make that first call before any stream
- *    capture begins on the device.
+ *  - The first call on each device looks up the buffer's device address (a set-up done
+ *    with that device current, repeated only if the device's context has changed since,
+ *    e.g. after cudaDeviceReset); make that first call before any stream capture begins on
+ *    the device.
  *  - All calls on a device share the one buffer; it is cleared at the start of every call,
  *    so leftover contents do not matter, but two calls that can run at the same time on
  *    the GPU (different streams, no ordering between them) race on it and give undefined
@@ -176,6 +183,27 @@ int streamkl_bwd_noalloc(int mode, const uint16_t* q1, const uint16_t* k1, const
                          const uint16_t* k2, const float* kl, const float* lse1, const float* lse2,
                          const float* dkl, int B, int Hq, int Hkv, int NQ, int NK, int d,
                          float scale, int causal, uint16_t* dq, uint16_t* dk, void* stream);
+
+/*
+ * Throughput probe of the two exponential paths the kernels use; no part of the KL
+ * computation.  The forward spends two exponentials per (row, key) pair with no second GEMM
+ * to amortise them (technical summary, "1. Formulação Online"), so their rate, not the
+ * tensor core, is its floor; this measures that rate.
+ *   kind 0: ex2.approx on the exponential unit (MUFU); kind 1: the FMA-pipe polynomial
+ *           the kernels evaluate part of their exponentials with.
+ *   iters : loop trips per thread (>= 1); the run takes about iters * 3 us (kind 0).
+ *   n_exp : if not NULL, receives the number of exponentials the launch evaluates
+ *           (4 CTAs per SM x 256 threads x 8 independent chains x iters).
+ * One kernel is launched on `stream`; the caller times it (CUDA events) and divides.
+ * Reads and writes no memory.  Returns STREAMKL_ERR_INVALID_ARG for a bad kind or iters.
+ */
+int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream);
+
+/*
+ * SM count of the current device, which the library's grid-sizing choices (key ranges of
+ * the split-K forward and of the backward) use; 148 (B200) when no device can be queried.
+ */
+int streamkl_num_sms(void);
 
 /* Static text for a status code (never NULL). */
 const char* streamkl_status_string(int status);

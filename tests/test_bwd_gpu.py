@@ -135,8 +135,9 @@ def sampled_check(name, mode, causal=None, heads_for_dk=1, rows_per_head=32, key
     gdq = dq.reshape(-1, d)[rows]
     e = rel_l2(gdq.reshape(w.B * w.Hq, rows_per_head, d)[None], odq.reshape(w.B * w.Hq, rows_per_head, d)[None], axes=(2, 3))
     assert e.max() <= GRAD_TOL, "%s dQ rel-L2 %.3g" % (name, e.max())
-    # dK: sampled keys of the first and last (b, KV head)
-    units = [0, w.B * w.Hkv - 1][:heads_for_dk] if heads_for_dk < 2 else [0, w.B * w.Hkv - 1]
+    # dK: sampled keys of the first (and, with heads_for_dk = 2, the last) (b, KV head): the
+    # first and last planes of the backward's grouped plane schedule
+    units = [0] if heads_for_dk < 2 else [0, w.B * w.Hkv - 1]
     keys = np.concatenate([u * w.NK + rng.choice(w.NK, keys_per_head, replace=False) for u in units])
     odk = oracle.bwd_dk_keys(mode, h["q1"], h["k1"], h["q2"], h["k2"], h["dkl"], keys,
                              scale=w.scale, causal=w.causal)
@@ -153,11 +154,11 @@ def test_full_size_b2h8n4k_mode1(causal):
 
 @pytest.mark.parametrize("mode", [1, 2])
 def test_full_size_headline(mode):
-    sampled_check("headline", mode, heads_for_dk=1)
+    sampled_check("headline", mode, heads_for_dk=2)
 
 
 def test_full_size_gqa_mode2():
-    sampled_check("gqa", 2, heads_for_dk=1, rows_per_head=16, keys_per_head=32)
+    sampled_check("gqa", 2, heads_for_dk=2, rows_per_head=16, keys_per_head=32)
 
 
 SIGN_CASES = [
@@ -173,10 +174,8 @@ SIGN_CASES = [
 @pytest.mark.parametrize("case", SIGN_CASES, ids=lambda c: "NQ%dNK%dd%d%s" % (c[3], c[4], c[5], "c" if c[6] else ""))
 def test_upstream_gradient_signs_and_zeros(case, kind, mode):
     """g of both signs takes the path that multiplies by g (a warp with any g < 0 cannot fold
-    log2 g into the exponent); g = 0 on every third row exercises the folded path's
-    log2 0 = -inf, which must leave those rows' dQ negligible: the exponential unit gives
-    exactly 0 there, the FMA-pipe exp2 (which clamps its argument at -126 to stay finite)
-    2^-126, so a zero row's dQ is at most of order 1e-36."""
+    log2 g into the exponent); g = 0 on every third row must give those rows exactly zero
+    dQ (their dS is zeroed, not computed from log2 0 = -inf)."""
     B, Hq, Hkv, NQ, NK, d, causal, shared = case
     w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=NQ + NK + d + 1)
     t = inputs.make(w, device="cuda")
@@ -196,7 +195,7 @@ def test_upstream_gradient_signs_and_zeros(case, kind, mode):
     check_grad(dq, odq, "%s %s dQ mode %d" % (case, kind, mode), zero_atol)
     check_grad(dk, odk, "%s %s dK mode %d" % (case, kind, mode), zero_atol)
     if kind == "zeros":
-        assert np.abs(dq[..., ::3, :]).max() <= 1e-30
+        assert np.abs(dq[..., ::3, :]).max() == 0.0
 
 
 def test_binding_refuses_mismatched_tensors_before_launch():
@@ -216,6 +215,16 @@ def test_binding_refuses_mismatched_tensors_before_launch():
     with pytest.raises(ValueError):
         binding.bwd(1, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"],
                     workspace=torch.empty(need // 4 - 1, device="cuda"))
+    # keys that disagree with the queries: a smaller batch, another head dim, a KV head count
+    # that does not divide the query heads -- each would size a tensor map past an allocation
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    for k in (torch.zeros(2, 2, 128, 64, **bf), torch.zeros(1, 2, 128, 32, **bf),
+              torch.zeros(1, 3, 128, 64, **bf)):
+        for call in (lambda: binding.fwd(t["q1"], k, t["q2"], k),
+                     lambda: binding.fwd_splitk(t["q1"], k, t["q2"], k),
+                     lambda: binding.bwd(1, t["q1"], k, t["q2"], k, kl, l1, l2, t["dkl"])):
+            with pytest.raises(ValueError):
+                call()
     w2 = inputs.custom(1, 2, 2, 1, 1024, 64, False, True, seed=4)     # 8 key tiles: a real split
     t2 = inputs.make(w2, device="cuda")
     assert binding.streamkl_fwd_splitk_workspace_bytes(1, 2, 1, 1024, 2) > 4
@@ -223,3 +232,23 @@ def test_binding_refuses_mismatched_tensors_before_launch():
         binding.fwd_splitk(t2["q1"], t2["k1"], t2["q2"], t2["k2"], splits=2,
                            workspace=torch.empty(1, device="cuda"))
     assert binding.streamkl_device_status() == binding.OK
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_reverse_kl_backward_by_swapping_the_distributions(mode):
+    """The gradient of KL(P2||P1): the same calls with the two distributions' arguments
+    swapped (forward, then backward with the swapped saved state), against the oracle's
+    backward on the swapped inputs.  Mode 1 then holds P2 fixed and trains (Q1, K1); mode 2
+    holds P1 fixed and trains (Q2, K2)."""
+    w = inputs.custom(1, 2, 2, 300, 300, 128, True, False, seed=43)
+    t = inputs.make(w, device="cuda")
+    t["dkl"] = torch.rand(t["dkl"].shape, generator=torch.Generator().manual_seed(5)).cuda() + 0.5
+    kl, l2, l1 = binding.fwd(t["q2"], t["k2"], t["q1"], t["k1"], scale=w.scale, causal=True)
+    dq, dk = binding.bwd(mode, t["q2"], t["k2"], t["q1"], t["k1"], kl, l2, l1, t["dkl"],
+                         scale=w.scale, causal=True)
+    assert binding.streamkl_device_status() == binding.OK
+    h = host(t)
+    odq, odk = oracle.bwd(mode, h["q2"], h["k2"], h["q1"], h["k1"], h["dkl"], scale=w.scale,
+                          causal=True)
+    check_grad(dq.cpu().double().numpy(), odq, "reverse KL dQ mode %d" % mode)
+    check_grad(dk.cpu().double().numpy(), odk, "reverse KL dK mode %d" % mode)
