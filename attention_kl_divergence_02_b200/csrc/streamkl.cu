@@ -14,6 +14,7 @@
 #include "streamkl.h"
 #include "sm100.cuh"
 #include "fwd_kernel.cuh"
+#include "fwd_keys_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "watchdog.cuh"
 #include "probe.cuh"
@@ -71,6 +72,7 @@ int make_map(CUtensorMap* map, const void* base, long long planes, long long row
 
 constexpr int kMaxDevices = 64;
 constexpr int kDefaultSMs = 148;   // B200; used only when no device can be queried
+constexpr int kKeysMaxRows = 8;    // query rows up to which the forward runs keys as MMA rows
 
 // SM count of the current device, looked up once per device ordinal (it cannot change while
 // the process runs).  The split heuristics size their grids in waves of one CTA per SM.
@@ -125,6 +127,26 @@ int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "streamkl_fwd launch");
     return STREAMKL_OK;
+}
+
+template <int D, bool SHARED, int ROWS>
+int launch_fwd_keys(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
+                    const CUtensorMap& k2, const skl::FwdParams& p, int grid, cudaStream_t st) {
+    auto kern = skl::streamkl_fwd_keys_kernel<D, SHARED, ROWS>;
+    constexpr int smem = skl::KeysCfg<D>::kSmem;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    kern<<<grid, skl::kKeysThreads, smem, st>>>(q1, q2, k1, k2, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "streamkl_fwd (few rows) launch");
+    return STREAMKL_OK;
+}
+
+template <int D, bool SHARED>
+int launch_fwd_keys_rows(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
+                         const CUtensorMap& k2, const skl::FwdParams& p, int grid, cudaStream_t st) {
+    return p.NQ == 1 ? launch_fwd_keys<D, SHARED, 1>(q1, q2, k1, k2, p, grid, st)
+                     : launch_fwd_keys<D, SHARED, 8>(q1, q2, k1, k2, p, grid, st);
 }
 
 // fp32 tile-blocked workspace -> bf16 rows (scale applied), one launch.
@@ -253,6 +275,40 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
     const bool shared = (k1 == k2);
     CUtensorMap mq1, mq2, mk1, mk2;
     int rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (NQ <= kKeysMaxRows) {
+        // at most 8 query rows: keys as the MMA's rows (16-row query boxes, rows past NQ zero)
+        if ((rc = make_map(&mq1, q1, (long long)B * Hq, NQ, d, 16))) return rc;
+        if ((rc = make_map(&mq2, q2, (long long)B * Hq, NQ, d, 16))) return rc;
+        if ((rc = make_map(&mk1, k1, (long long)B * Hkv, NK, d))) return rc;
+        if ((rc = make_map(&mk2, k2, (long long)B * Hkv, NK, d))) return rc;
+        skl::FwdParams p;
+        p.rep4 = 0;
+        p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NQ = NQ; p.NK = NK;
+        p.causal = causal ? 1 : 0;
+        p.n_qblk = 1;
+        p.sl2 = scale * 1.4426950408889634f;
+        p.scale = scale;
+        p.kl = kl; p.lse1 = lse1; p.lse2 = lse2;
+        split_ranges(NK, splits, &p.kps, &p.splits);
+        p.part = p.splits > 1 ? part : nullptr;
+        const long long grid = (long long)B * Hq * p.splits;
+        if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
+        if (d == 128) {
+            rc = shared ? launch_fwd_keys_rows<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                        : launch_fwd_keys_rows<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+        } else {
+            rc = shared ? launch_fwd_keys_rows<64, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
+                        : launch_fwd_keys_rows<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
+        }
+        if (rc || p.splits == 1) return rc;
+        const long long R = (long long)B * Hq * NQ;
+        const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * num_sms());
+        skl::streamkl_splitk_merge_kernel<<<mgrid, 256, 0, st>>>(part, p.splits, R, scale, kl, lse1, lse2);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+        return STREAMKL_OK;
+    }
     // at most 32 query rows: they are loaded once into each 32-lane quarter of the query
     // tile (32-row boxes), so that all four warps of a warpgroup can fold them
     const int rep4 = NQ <= 32 ? 1 : 0;
@@ -272,7 +328,6 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
     p.part = p.splits > 1 ? part : nullptr;
     const long long grid = (long long)B * Hq * p.n_qblk * p.splits;
     if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128) {
         rc = shared ? launch_fwd<128, true>(mq1, mq2, mk1, mk2, p, (int)grid, st)
                     : launch_fwd<128, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
@@ -308,6 +363,16 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
 
 int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
     if (B < 1 || Hq < 1 || NQ < 1 || NK < 1) return 1;
+    if (NQ <= kKeysMaxRows) {
+        // keys as MMA rows: one wave of two CTAs per SM, every CTA streaming its key range
+        const long long heads = (long long)B * Hq;
+        const int nkt = (NK + 127) / 128;
+        const long long want = (2ll * num_sms()) / heads;
+        if (want <= 1 || nkt < 2) return 1;
+        int kps, used;
+        split_ranges(NK, (int)std::min<long long>(want, nkt), &kps, &used);
+        return used;
+    }
     const long long blocks = (long long)B * Hq * ((NQ + 255) / 256);
     const int nkt = (NK + 127) / 128;
     const int sms = num_sms();

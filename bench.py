@@ -623,7 +623,7 @@ def run_decode(args):
                    "splits": splits, "bytes_per_step": nbytes,
                    "l2": "keys (537 MB) larger than the 126 MB L2; no flush"},
         "unsplit_ms": u_ms, "speedup_vs_unsplit": u_ms / s_ms,
-        "roofline": {"bound": "hbm", "kernel": "streamkl_fwd_kernel (split) + merge",
+        "roofline": {"bound": "hbm", "kernel": "streamkl_fwd_keys_kernel (split, keys as MMA rows) + merge",
                      "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                      "traffic": None, "peak_source": "%s hbm_gbs" % peak_src,
                      "note": "achieved = algorithmic bytes per step / CUDA-event time of the step"},

@@ -130,10 +130,15 @@ def test_splitk_workspace_and_choice(lib):
     # the library's choice: none when the query blocks fill the GPU, several otherwise
     assert binding.streamkl_fwd_splits(1, 32, 16384, 16384) == 1
     assert binding.streamkl_fwd_splits(1, 1, 1, 128) == 1
-    assert binding.streamkl_fwd_splits(4, 32, 1, 32768) == 1     # 128 blocks fill the GPU
+    # at most 8 query rows (keys as MMA rows, two CTAs per SM): one wave of 2 x 148 CTAs
+    assert binding.streamkl_fwd_splits(4, 32, 1, 32768) == 2     # 128 heads -> 256 CTAs
+    assert binding.streamkl_fwd_splits(8, 40, 1, 32768) == 1     # 320 heads fill the wave
     s = binding.streamkl_fwd_splits(1, 16, 1, 131072)
-    assert 4 <= s <= 64
+    assert s == 18                                               # 16 x 18 = 288 CTAs
     assert binding.streamkl_fwd_splitk_workspace_bytes(1, 16, 1, 131072, 0) == s * 5 * 16 * 4
+    # more rows: the query-block kernel's model (waves x (tiles per range + 8))
+    s = binding.streamkl_fwd_splits(1, 16, 32, 131072)
+    assert 4 <= s <= 64
 
 
 def splitk_call(**kw):

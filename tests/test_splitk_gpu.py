@@ -47,6 +47,32 @@ def test_matches_oracle(case):
     check_fwd(_split(t, w, splits), _oracle(t, w), "splitk %s" % (case,))
 
 
+FEW_ROWS = [
+    # B, Hq, Hkv, NQ, NK, d, causal, shared, splits  (at most 8 query rows: keys as MMA rows)
+    (1, 3, 3, 2, 700, 128, False, True, 0),
+    (2, 4, 2, 8, 1000, 64, False, False, 0),      # GQA, distinct keys
+    (1, 2, 2, 5, 5, 128, True, True, 1),          # causal (NQ == NK), one tile
+    (1, 2, 2, 8, 8, 64, True, False, 3),          # causal, more ranges asked than tiles
+    (1, 1, 1, 3, 129, 128, False, False, 1),      # one range, a ragged second key tile
+    (1, 4, 1, 7, 4000, 128, False, True, 5),      # GQA 4:1, shared keys
+    (1, 2, 2, 1, 300, 64, False, True, 0),
+]
+
+
+@pytest.mark.parametrize("case", FEW_ROWS, ids=lambda c: "B%dHq%dHkv%dNQ%dNK%dd%d%s%s_s%d" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "", "sh" if c[7] else "", c[8]))
+def test_few_rows_matches_oracle(case):
+    """At most 8 query rows: split and unsplit forward against the oracle."""
+    B, Hq, Hkv, NQ, NK, d, causal, shared, splits = case
+    w = inputs.custom(B, Hq, Hkv, NQ, NK, d, causal, shared, seed=11 + NQ + NK + d)
+    t = inputs.make(w, device="cuda")
+    want = _oracle(t, w)
+    check_fwd(_split(t, w, splits), want, "few rows split %s" % (case,))
+    got = binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=w.causal)
+    assert binding.streamkl_device_status() == binding.OK
+    check_fwd(tuple(x.cpu().double().numpy() for x in got), want, "few rows unsplit %s" % (case,))
+
+
 def test_matches_unsplit_forward():
     w = inputs.custom(2, 4, 4, 64, 4096, 128, False, True, seed=11)
     t = inputs.make(w, device="cuda")
