@@ -24,6 +24,7 @@ ERR_TIMEOUT = 4
 
 EXPORTS = (
     "streamkl_fwd",
+    "streamkl_fwd_sym",
     "streamkl_fwd_splitk",
     "streamkl_fwd_splits",
     "streamkl_fwd_splitk_workspace_bytes",
@@ -64,6 +65,8 @@ def load(path=None):
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.streamkl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
     lib.streamkl_fwd.restype = i
+    lib.streamkl_fwd_sym.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp, vp]
+    lib.streamkl_fwd_sym.restype = i
     lib.streamkl_fwd_splitk.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp, vp, vp, vp, sz, vp]
     lib.streamkl_fwd_splitk.restype = i
     lib.streamkl_fwd_splits.argtypes = [i, i, i, i]
@@ -119,6 +122,13 @@ def streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, kl, lse1,
     return load().streamkl_fwd(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), B, Hq, Hkv, NQ, NK, d,
                                float(scale), int(bool(causal)), _ptr(kl), _ptr(lse1), _ptr(lse2),
                                _stream(stream))
+
+
+def streamkl_fwd_sym(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, kl12, kl21, lse1, lse2,
+                     stream=None):
+    return load().streamkl_fwd_sym(_ptr(q1), _ptr(k1), _ptr(q2), _ptr(k2), B, Hq, Hkv, NQ, NK, d,
+                                   float(scale), int(bool(causal)), _ptr(kl12), _ptr(kl21), _ptr(lse1),
+                                   _ptr(lse2), _stream(stream))
 
 
 def streamkl_fwd_splitk(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, kl, lse1, lse2,
@@ -257,6 +267,23 @@ def fwd(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
     rc = streamkl_fwd(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, *out, stream=stream)
     if rc != OK:
         raise StreamKLError(rc, "streamkl_fwd")
+    return out
+
+
+def fwd_sym(q1, k1, q2, k2, scale=None, causal=False, out=None, stream=None):
+    """Returns (kl12, kl21, lse1, lse2), fp32 [B,Hq,NQ]: KL(P1||P2), KL(P2||P1) and both LSEs in
+    one pass over the keys; kl12 + kl21 is the symmetric divergence."""
+    import torch
+    _check_inputs(q1, k1, q2, k2)
+    B, Hq, Hkv, NQ, NK, d = _dims(q1, k1)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = tuple(torch.empty((B, Hq, NQ), dtype=torch.float32, device=q1.device) for _ in range(4))
+    for name, o in zip(("kl12", "kl21", "lse1", "lse2"), out):
+        _check_tensor(name, o, (B, Hq, NQ), torch.float32, q1.device)
+    rc = streamkl_fwd_sym(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, *out, stream=stream)
+    if rc != OK:
+        raise StreamKLError(rc, "streamkl_fwd_sym")
     return out
 
 

@@ -48,6 +48,7 @@ struct FwdParams {
     int splits;    // key ranges per query block (1 = no split)
     int kps;       // key tiles per range
     float* part;   // splits > 1: partial state [splits][5][B*Hq*NQ]: m1, l1, m2, l2, acc
+    float* kl21;   // symmetric variant only: KL(P2 || P1) per row (else unused)
 };
 
 constexpr int kFwdThreads = 384;
@@ -95,9 +96,14 @@ constexpr uint32_t kEmu2 = SKL_FWD_EMU2;
 // Fold 32 columns of one row, all valid keys, into the running scalars (x = S1 raw
 // scores, y = S2 raw).  Adjacent columns are processed as fp32x2 pairs: they are adjacent
 // registers of one TMEM load, so each add/FMA instruction serves two columns.
+//
+// SYM: also accumulate acc2 = sum 2^(u2 - m2) (s1 - s2), rescaled with m2, whose negation over
+// l2 is the reverse direction's (s2 - s1) term, so that one pass gives both KL(P1 || P2) and
+// KL(P2 || P1) (their sum is the symmetric divergence).
+template <bool SYM>
 __device__ __forceinline__ void fold_chunk_full(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
                                                 float sl2, float& m1, float& l1, float& m2,
-                                                float& l2, float& acc) {
+                                                float& l2, float& acc, float& acc2) {
     float mx1 = __uint_as_float(xa[0]), mx2 = __uint_as_float(ya[0]);
 #pragma unroll
     for (int k = 1; k < 31; k += 2) {
@@ -119,6 +125,7 @@ __device__ __forceinline__ void fold_chunk_full(const uint32_t (&xa)[32], const 
     float2 L1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float2 L2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float2 AC[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 AC2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int pr = 0; pr < 16; ++pr) {
         const float2 xk = make_float2(__uint_as_float(xa[2 * pr]), __uint_as_float(xa[2 * pr + 1]));
@@ -131,6 +138,7 @@ __device__ __forceinline__ void fold_chunk_full(const uint32_t (&xa)[32], const 
         L2[pr & 1] = __fadd2_rn(L2[pr & 1], e2);
         const float2 dk = __ffma2_rn(yk, neg1, xk);
         AC[pr & 1] = __ffma2_rn(e1, dk, AC[pr & 1]);
+        if (SYM) AC2[pr & 1] = __ffma2_rn(e2, dk, AC2[pr & 1]);
     }
     const float2 L1s = __fadd2_rn(L1[0], L1[1]);
     const float2 L2s = __fadd2_rn(L2[0], L2[1]);
@@ -138,13 +146,18 @@ __device__ __forceinline__ void fold_chunk_full(const uint32_t (&xa)[32], const 
     l1 = fmaf(l1, a1, L1s.x + L1s.y);
     acc = fmaf(acc, a1, ACs.x + ACs.y);
     l2 = fmaf(l2, a2, L2s.x + L2s.y);
+    if (SYM) {
+        const float2 AC2s = __fadd2_rn(AC2[0], AC2[1]);
+        acc2 = fmaf(acc2, a2, AC2s.x + AC2s.y);
+    }
 }
 
 // Same fold for a chunk with invalid columns (bit k of `valid` clear): those are left out of
 // the maxima and of every sum, including the (s1 - s2) term, which would be NaN there.
+template <bool SYM>
 __device__ __forceinline__ void fold_chunk_masked(const uint32_t (&xa)[32], const uint32_t (&ya)[32],
                                                   uint32_t valid, float sl2, float& m1, float& l1,
-                                                  float& m2, float& l2, float& acc) {
+                                                  float& m2, float& l2, float& acc, float& acc2) {
     float x[32], y[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
@@ -164,7 +177,7 @@ __device__ __forceinline__ void fold_chunk_masked(const uint32_t (&xa)[32], cons
     const float a2 = ex2(m2 - m2n);
     m1 = m1n;
     m2 = m2n;
-    float sl1 = 0.f, sl2v = 0.f, sac = 0.f;
+    float sl1 = 0.f, sl2v = 0.f, sac = 0.f, sac2 = 0.f;
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
         const float e1 = ex2(fmaf(x[k], sl2, -m1n));
@@ -173,13 +186,15 @@ __device__ __forceinline__ void fold_chunk_masked(const uint32_t (&xa)[32], cons
         sl1 += e1;
         sl2v += e2;
         sac = fmaf(e1, diff, sac);
+        if (SYM) sac2 = fmaf(e2, diff, sac2);
     }
     l1 = fmaf(l1, a1, sl1);
     acc = fmaf(acc, a1, sac);
     l2 = fmaf(l2, a2, sl2v);
+    if (SYM) acc2 = fmaf(acc2, a2, sac2);
 }
 
-template <int D, bool SHARED_K>
+template <int D, bool SHARED_K, bool SYM>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
@@ -389,7 +404,8 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         const int c_lo = rep4 ? quarter : 0;
         const int c_hi = rep4 ? quarter + 1 : 4;
         // writes one finished row: its partial state (split-K) or KL, LSE1, LSE2
-        auto write_row = [&](int i, float m1, float l1, float m2, float l2, float acc) {
+        constexpr int kF = SYM ? 6 : 5;   // fields of a row's state in the merge buffers
+        auto write_row = [&](int i, float m1, float l1, float m2, float l2, float acc, float acc2) {
             if (p.splits > 1) {
                 const size_t R = (size_t)p.B * p.Hq * p.NQ;
                 float* dst = p.part + (size_t)sp * 5 * R + (size_t)bh * p.NQ + i;
@@ -406,15 +422,17 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 p.lse1[o] = (m1 + lg1) * LN2;
                 p.lse2[o] = (m2 + lg2) * LN2;
                 p.kl[o] = p.scale * acc / l1 + ((m2 - m1) + (lg2 - lg1)) * LN2;
+                if (SYM) p.kl21[o] = -p.scale * acc2 / l2 + ((m1 - m2) + (lg1 - lg2)) * LN2;
             }
         };
         if (split && g < 2) {
             const float sl2 = p.sl2;
             const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
-            float st[2][5];
+            float st[2][6];
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2) {
                 st[t2][0] = -1e30f; st[t2][1] = 0.f; st[t2][2] = -1e30f; st[t2][3] = 0.f; st[t2][4] = 0.f;
+                st[t2][5] = 0.f;
             }
             bool ok = true;
             for (int j = j0; j < nj && ok; ++j) {
@@ -447,15 +465,16 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                             mbar_arrive(BAR(C::S_FREE + t2));
                         }
                         if (!masked) {
-                            fold_chunk_full(xa, ya, sl2, st[t2][0], st[t2][1], st[t2][2], st[t2][3], st[t2][4]);
+                            fold_chunk_full<SYM>(xa, ya, sl2, st[t2][0], st[t2][1], st[t2][2], st[t2][3],
+                                                 st[t2][4], st[t2][5]);
                         } else {
                             const int k0 = kb + c * 32;
                             int lim = p.NK - k0;
                             if (p.causal) lim = min(lim, i2 - k0 + 1);
                             const uint32_t valid = lim >= 32 ? 0xFFFFFFFFu
                                                  : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-                            fold_chunk_masked(xa, ya, valid, sl2, st[t2][0], st[t2][1], st[t2][2],
-                                              st[t2][3], st[t2][4]);
+                            fold_chunk_masked<SYM>(xa, ya, valid, sl2, st[t2][0], st[t2][1], st[t2][2],
+                                                   st[t2][3], st[t2][4], st[t2][5]);
                         }
                     }
                 }
@@ -467,14 +486,14 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2)
 #pragma unroll
-                for (int f = 0; f < 5; ++f) mb[((t2 * 2 + g) * 5 + f) * 128 + r] = st[t2][f];
+                for (int f = 0; f < kF; ++f) mb[((t2 * 2 + g) * kF + f) * 128 + r] = st[t2][f];
             mbar_arrive(BAR(C::MERGE));
             if (g == 0) {
                 ok = mbar_wait(BAR(C::MERGE), 0, abort_flag) && ok;
 #pragma unroll
                 for (int t2 = 0; t2 < 2; ++t2) {
-                    const float* a0 = mb + (t2 * 2 + 0) * 5 * 128 + r;
-                    const float* a1 = mb + (t2 * 2 + 1) * 5 * 128 + r;
+                    const float* a0 = mb + (t2 * 2 + 0) * kF * 128 + r;
+                    const float* a1 = mb + (t2 * 2 + 1) * kF * 128 + r;
                     const float M1 = fmaxf(a0[0], a1[0]);
                     const float M2 = fmaxf(a0[2 * 128], a1[2 * 128]);
                     const float e10 = ex2(a0[0] - M1), e11 = ex2(a1[0] - M1);
@@ -482,8 +501,9 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     const float L1 = fmaf(a0[128], e10, a1[128] * e11);
                     const float A = fmaf(a0[4 * 128], e10, a1[4 * 128] * e11);
                     const float L2 = fmaf(a0[3 * 128], e20, a1[3 * 128] * e21);
+                    const float A2 = SYM ? fmaf(a0[5 * 128], e20, a1[5 * 128] * e21) : 0.f;
                     const int i2 = q0[t2] + r;
-                    if (ok && i2 < p.NQ) write_row(i2, M1, L1, M2, L2, A);
+                    if (ok && i2 < p.NQ) write_row(i2, M1, L1, M2, L2, A, A2);
                 }
             }
         } else if (!split && g < (alt ? 2 : ntiles)) {
@@ -491,7 +511,7 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             const uint32_t tS1 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * 256);
             const uint32_t tS2 = tS1 + 128;
             const float sl2 = p.sl2;
-            float m1 = -1e30f, l1 = 0.f, m2 = -1e30f, l2 = 0.f, acc = 0.f;
+            float m1 = -1e30f, l1 = 0.f, m2 = -1e30f, l2 = 0.f, acc = 0.f, acc2 = 0.f;
             bool ok = true;
             // a warp whose 32 rows all lie past NQ only keeps the barrier protocol
             const bool any_row = rep4 || q0[t] + quarter * 32 < p.NQ;
@@ -520,14 +540,14 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                         mbar_arrive(BAR(C::S_FREE + g));
                     }
                     if (!masked) {
-                        fold_chunk_full(xa, ya, sl2, m1, l1, m2, l2, acc);
+                        fold_chunk_full<SYM>(xa, ya, sl2, m1, l1, m2, l2, acc, acc2);
                     } else {
                         const int k0 = kb + c * 32;
                         int lim = p.NK - k0;                       // keys k0 + k valid if k < lim
                         if (p.causal) lim = min(lim, i - k0 + 1);  // ... and k0 + k <= i
                         const uint32_t valid = lim >= 32 ? 0xFFFFFFFFu
                                              : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-                        fold_chunk_masked(xa, ya, valid, sl2, m1, l1, m2, l2, acc);
+                        fold_chunk_masked<SYM>(xa, ya, valid, sl2, m1, l1, m2, l2, acc, acc2);
                     }
                 }
             }
@@ -540,31 +560,32 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 const int rows_per = rep4 ? 32 : 128;
                 const int rho = rep4 ? lane : r;
                 const int kappa = (alt ? g : 0) * (rep4 ? 4 : 1) + (rep4 ? quarter : 0);
-                const float st[5] = {m1, l1, m2, l2, acc};
+                const float st[6] = {m1, l1, m2, l2, acc, acc2};
 #pragma unroll
-                for (int f = 0; f < 5; ++f) mb[(kappa * 5 + f) * rows_per + rho] = st[f];
+                for (int f = 0; f < kF; ++f) mb[(kappa * kF + f) * rows_per + rho] = st[f];
                 mbar_arrive(BAR(C::MERGE));
                 if (g == 0 && (!rep4 || quarter == 0)) {
                     ok = mbar_wait(BAR(C::MERGE), 0, abort_flag) && ok;
                     float M1 = -1e30f, M2 = -1e30f;
                     for (int w = 0; w < n_contrib; ++w) {
-                        M1 = fmaxf(M1, mb[(w * 5 + 0) * rows_per + rho]);
-                        M2 = fmaxf(M2, mb[(w * 5 + 2) * rows_per + rho]);
+                        M1 = fmaxf(M1, mb[(w * kF + 0) * rows_per + rho]);
+                        M2 = fmaxf(M2, mb[(w * kF + 2) * rows_per + rho]);
                     }
-                    float L1 = 0.f, L2 = 0.f, A = 0.f;
+                    float L1 = 0.f, L2 = 0.f, A = 0.f, A2 = 0.f;
                     for (int w = 0; w < n_contrib; ++w) {
-                        const float a1 = ex2(mb[(w * 5 + 0) * rows_per + rho] - M1);
-                        const float a2 = ex2(mb[(w * 5 + 2) * rows_per + rho] - M2);
-                        L1 = fmaf(mb[(w * 5 + 1) * rows_per + rho], a1, L1);
-                        A = fmaf(mb[(w * 5 + 4) * rows_per + rho], a1, A);
-                        L2 = fmaf(mb[(w * 5 + 3) * rows_per + rho], a2, L2);
+                        const float a1 = ex2(mb[(w * kF + 0) * rows_per + rho] - M1);
+                        const float a2 = ex2(mb[(w * kF + 2) * rows_per + rho] - M2);
+                        L1 = fmaf(mb[(w * kF + 1) * rows_per + rho], a1, L1);
+                        A = fmaf(mb[(w * kF + 4) * rows_per + rho], a1, A);
+                        L2 = fmaf(mb[(w * kF + 3) * rows_per + rho], a2, L2);
+                        if (SYM) A2 = fmaf(mb[(w * kF + 5) * rows_per + rho], a2, A2);
                     }
-                    m1 = M1; l1 = L1; m2 = M2; l2 = L2; acc = A;
+                    m1 = M1; l1 = L1; m2 = M2; l2 = L2; acc = A; acc2 = A2;
                 } else {
                     ok = false;   // one thread per row writes it
                 }
             }
-            if (ok && i < p.NQ) write_row(i, m1, l1, m2, l2, acc);
+            if (ok && i < p.NQ) write_row(i, m1, l1, m2, l2, acc, acc2);
         }
     }
 

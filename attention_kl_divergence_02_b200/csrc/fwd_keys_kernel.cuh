@@ -35,8 +35,8 @@ struct KeysCfg {
     static constexpr int kSlots = (D == 128) ? 3 : 6;
     static constexpr int kQ = 0;                            // Q box b at kQ + b*kQBox
     static constexpr int kK = 8192;                         // key slot s at kK + s*kTile
-    static constexpr int kMerge = kK + kSlots * kTile;      // 4 warps x 8 rows x 5 floats
-    static constexpr int kBar = kMerge + 4 * 8 * 5 * 4;
+    static constexpr int kMerge = kK + kSlots * kTile;      // 4 warps x 8 rows x 6 floats
+    static constexpr int kBar = kMerge + 4 * 8 * 6 * 4;
     static constexpr int Q_FULL = 0;
     static constexpr int K_FULL = 1;                        // + s
     static constexpr int K_EMPTY = 1 + kSlots;              // + s
@@ -50,9 +50,11 @@ struct KeysCfg {
 };
 
 // One online step of a lane's state for one query row and one key (base-2 scores s1, s2 =
-// raw * scale * log2 e; diff = raw s1 - raw s2).
+// raw * scale * log2 e; diff = raw s1 - raw s2).  SYM: also acc2, the same sum weighted by
+// P2 and rescaled with m2 (the reverse direction's term, negated).
+template <bool SYM>
 __device__ __forceinline__ void keys_update(float s1, float s2, float diff, float& m1, float& l1,
-                                            float& m2, float& l2, float& acc) {
+                                            float& m2, float& l2, float& acc, float& acc2) {
     const float n1 = fmaxf(m1, s1);
     const float n2 = fmaxf(m2, s2);
     const float a1 = ex2(m1 - n1), e1 = ex2(s1 - n1);
@@ -60,24 +62,28 @@ __device__ __forceinline__ void keys_update(float s1, float s2, float diff, floa
     l1 = fmaf(l1, a1, e1);
     acc = fmaf(acc, a1, e1 * diff);
     l2 = fmaf(l2, a2, e2);
+    if (SYM) acc2 = fmaf(acc2, a2, e2 * diff);
     m1 = n1;
     m2 = n2;
 }
 
 // Combines state b into state a (both over disjoint key sets).
+template <bool SYM>
 __device__ __forceinline__ void keys_combine(float& m1, float& l1, float& m2, float& l2, float& acc,
-                                             float bm1, float bl1, float bm2, float bl2, float bacc) {
+                                             float& acc2, float bm1, float bl1, float bm2, float bl2,
+                                             float bacc, float bacc2) {
     const float M1 = fmaxf(m1, bm1), M2 = fmaxf(m2, bm2);
     const float ea = ex2(m1 - M1), eb = ex2(bm1 - M1);
     const float fa = ex2(m2 - M2), fb = ex2(bm2 - M2);
     l1 = fmaf(l1, ea, bl1 * eb);
     acc = fmaf(acc, ea, bacc * eb);
     l2 = fmaf(l2, fa, bl2 * fb);
+    if (SYM) acc2 = fmaf(acc2, fa, bacc2 * fb);
     m1 = M1;
     m2 = M2;
 }
 
-template <int D, bool SHARED_K, int ROWS>
+template <int D, bool SHARED_K, int ROWS, bool SYM>
 __global__ void __launch_bounds__(kKeysThreads, 2)
 streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                          const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
@@ -224,10 +230,10 @@ streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_
         const int r = quarter * 32 + lane;                  // key lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.sl2;
-        float m1[ROWS], l1[ROWS], m2[ROWS], l2[ROWS], acc[ROWS];
+        float m1[ROWS], l1[ROWS], m2[ROWS], l2[ROWS], acc[ROWS], acc2[ROWS];
 #pragma unroll
         for (int t = 0; t < ROWS; ++t) {
-            m1[t] = -1e30f; l1[t] = 0.f; m2[t] = -1e30f; l2[t] = 0.f; acc[t] = 0.f;
+            m1[t] = -1e30f; l1[t] = 0.f; m2[t] = -1e30f; l2[t] = 0.f; acc[t] = 0.f; acc2[t] = 0.f;
         }
         bool ok = true;
         for (int u = 0; u < nj; ++u) {
@@ -249,7 +255,7 @@ streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_
                 for (int t = 0; t < ROWS; ++t) {
                     if (t < p.NQ && (!p.causal || key <= t)) {
                         const float x = __uint_as_float(xa[t]), y = __uint_as_float(ya[t]);
-                        keys_update(x * sl2, y * sl2, x - y, m1[t], l1[t], m2[t], l2[t], acc[t]);
+                        keys_update<SYM>(x * sl2, y * sl2, x - y, m1[t], l1[t], m2[t], l2[t], acc[t], acc2[t]);
                     }
                 }
             }
@@ -264,15 +270,16 @@ streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_
                 const float bm2 = __shfl_xor_sync(0xffffffffu, m2[t], o);
                 const float bl2 = __shfl_xor_sync(0xffffffffu, l2[t], o);
                 const float bac = __shfl_xor_sync(0xffffffffu, acc[t], o);
-                keys_combine(m1[t], l1[t], m2[t], l2[t], acc[t], bm1, bl1, bm2, bl2, bac);
+                const float bac2 = SYM ? __shfl_xor_sync(0xffffffffu, acc2[t], o) : 0.f;
+                keys_combine<SYM>(m1[t], l1[t], m2[t], l2[t], acc[t], acc2[t], bm1, bl1, bm2, bl2, bac, bac2);
             }
         }
-        float* mb = reinterpret_cast<float*>(smem + C::kMerge);   // [warp][row][5]
+        float* mb = reinterpret_cast<float*>(smem + C::kMerge);   // [warp][row][6]
         if (lane == 0) {
 #pragma unroll
             for (int t = 0; t < ROWS; ++t) {
-                float* e = mb + (quarter * 8 + t) * 5;
-                e[0] = m1[t]; e[1] = l1[t]; e[2] = m2[t]; e[3] = l2[t]; e[4] = acc[t];
+                float* e = mb + (quarter * 8 + t) * 6;
+                e[0] = m1[t]; e[1] = l1[t]; e[2] = m2[t]; e[3] = l2[t]; e[4] = acc[t]; e[5] = acc2[t];
             }
             mbar_arrive(BAR(C::MERGE));
         }
@@ -280,10 +287,10 @@ streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_
             ok = mbar_wait(BAR(C::MERGE), 0, abort_flag) && ok;
             const int t = lane;
             if (ok && t < ROWS && t < p.NQ) {
-                float M1 = -1e30f, L1 = 0.f, M2 = -1e30f, L2 = 0.f, A = 0.f;
+                float M1 = -1e30f, L1 = 0.f, M2 = -1e30f, L2 = 0.f, A = 0.f, A2 = 0.f;
                 for (int w = 0; w < 4; ++w) {
-                    const float* e = mb + (w * 8 + t) * 5;
-                    keys_combine(M1, L1, M2, L2, A, e[0], e[1], e[2], e[3], e[4]);
+                    const float* e = mb + (w * 8 + t) * 6;
+                    keys_combine<SYM>(M1, L1, M2, L2, A, A2, e[0], e[1], e[2], e[3], e[4], e[5]);
                 }
                 const size_t o = (size_t)bh * p.NQ + t;
                 if (p.splits > 1) {
@@ -300,6 +307,7 @@ streamkl_fwd_keys_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_
                     p.lse1[o] = (M1 + lg1) * LN2;
                     p.lse2[o] = (M2 + lg2) * LN2;
                     p.kl[o] = p.scale * A / L1 + ((M2 - M1) + (lg2 - lg1)) * LN2;
+                    if (SYM) p.kl21[o] = -p.scale * A2 / L2 + ((M1 - M2) + (lg1 - lg2)) * LN2;
                 }
             }
         }

@@ -119,7 +119,7 @@ int set_smem(K kernel, int bytes) {
 template <int D, bool SHARED>
 int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                const CUtensorMap& k2, const skl::FwdParams& p, int grid, cudaStream_t st) {
-    auto kern = skl::streamkl_fwd_kernel<D, SHARED>;
+    auto kern = p.kl21 ? skl::streamkl_fwd_kernel<D, SHARED, true> : skl::streamkl_fwd_kernel<D, SHARED, false>;
     constexpr int smem = skl::FwdCfg<D>::kSmem;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
@@ -132,7 +132,8 @@ int launch_fwd(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& 
 template <int D, bool SHARED, int ROWS>
 int launch_fwd_keys(const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                     const CUtensorMap& k2, const skl::FwdParams& p, int grid, cudaStream_t st) {
-    auto kern = skl::streamkl_fwd_keys_kernel<D, SHARED, ROWS>;
+    auto kern = p.kl21 ? skl::streamkl_fwd_keys_kernel<D, SHARED, ROWS, true>
+                       : skl::streamkl_fwd_keys_kernel<D, SHARED, ROWS, false>;
     constexpr int smem = skl::KeysCfg<D>::kSmem;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
@@ -269,9 +270,10 @@ void split_ranges(int NK, int splits, int* kps, int* used) {
     *used = (nkt + *kps - 1) / *kps;
 }
 
+// kl21 != nullptr: the symmetric variant (also KL(P2 || P1) per row), one key range only.
 int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2, int B,
              int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal, int splits, float* kl,
-             float* lse1, float* lse2, float* part, void* stream) {
+             float* lse1, float* lse2, float* part, float* kl21, void* stream) {
     const bool shared = (k1 == k2);
     CUtensorMap mq1, mq2, mk1, mk2;
     int rc;
@@ -290,6 +292,7 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
         p.sl2 = scale * 1.4426950408889634f;
         p.scale = scale;
         p.kl = kl; p.lse1 = lse1; p.lse2 = lse2;
+        p.kl21 = kl21;
         split_ranges(NK, splits, &p.kps, &p.splits);
         p.part = p.splits > 1 ? part : nullptr;
         const long long grid = (long long)B * Hq * p.splits;
@@ -324,6 +327,7 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
     p.sl2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.kl = kl; p.lse1 = lse1; p.lse2 = lse2;
+    p.kl21 = kl21;
     split_ranges(NK, splits, &p.kps, &p.splits);
     p.part = p.splits > 1 ? part : nullptr;
     const long long grid = (long long)B * Hq * p.n_qblk * p.splits;
@@ -358,7 +362,20 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
         !aligned16(lse1) || !aligned16(lse2))
         return STREAMKL_ERR_UNSUPPORTED;
     return fwd_impl(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, 1, kl, lse1, lse2,
-                    nullptr, stream);
+                    nullptr, nullptr, stream);
+}
+
+int streamkl_fwd_sym(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
+                     int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                     float* kl12, float* kl21, float* lse1, float* lse2, void* stream) {
+    if (!q1 || !k1 || !q2 || !k2 || !kl12 || !kl21 || !lse1 || !lse2) return STREAMKL_ERR_INVALID_ARG;
+    int rc = check_shape(B, Hq, Hkv, NQ, NK, d, scale, causal);
+    if (rc) return rc;
+    const void* ptrs[] = {q1, k1, q2, k2, kl12, kl21, lse1, lse2};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return STREAMKL_ERR_UNSUPPORTED;
+    return fwd_impl(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, 1, kl12, lse1, lse2,
+                    nullptr, kl21, stream);
 }
 
 int streamkl_fwd_splits(int B, int Hq, int NQ, int NK) {
@@ -426,7 +443,7 @@ int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* 
     const size_t need = streamkl_fwd_splitk_workspace_bytes(B, Hq, NQ, NK, splits);
     if (need > 0 && (!workspace || workspace_bytes < need)) return STREAMKL_ERR_INVALID_ARG;
     return fwd_impl(q1, k1, q2, k2, B, Hq, Hkv, NQ, NK, d, scale, causal, splits, kl, lse1, lse2,
-                    static_cast<float*>(workspace), stream);
+                    static_cast<float*>(workspace), nullptr, stream);
 }
 
 }  // extern "C"

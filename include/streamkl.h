@@ -69,6 +69,22 @@ int streamkl_fwd(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, con
                  float* kl, float* lse1, float* lse2, void* stream);
 
 /*
+ * Both directions in one pass: KL(P1 || P2) and KL(P2 || P1) per query row, whose sum is the
+ * symmetric (Jeffreys) divergence.  The pages only outline that fused online primitives
+ * extend to other coupled two-distribution reductions (technical summary, "Significância");
+ * this is the plainest such extension: the forward's five running scalars plus a sixth,
+ * acc2 = sum_j exp(s2_j - m2) (s1_j - s2_j), rescaled like l2 whenever m2 grows, so that
+ * KL(P2 || P1) = -acc2/l2 + LSE1 - LSE2.  The keys are read once for both directions.
+ *
+ *   kl12, kl21, lse1, lse2 : fp32 [B,Hq,NQ] outputs, overwritten (natural-log units).
+ * Other arguments, errors and ownership as streamkl_fwd.  No key-range split (one CTA per query
+ * block, or per head for at most 8 rows); extra device memory: none.
+ */
+int streamkl_fwd_sym(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2,
+                     int B, int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal,
+                     float* kl12, float* kl21, float* lse1, float* lse2, void* stream);
+
+/*
  * Forward with the key tiles split into ranges, for few query rows and many keys (the
  * decoding case the technical summary's "3. Otimizações de Kernel de GPU" names for split-K):
  * each (query block, key range) is one CTA, so B*Hq*ceil(NQ/256) blocks that would leave
@@ -92,9 +108,11 @@ int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* 
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The number of key ranges streamkl_fwd_splitk uses for splits = 0: 1 when the query blocks
- * alone fill the GPU, else the fewest ranges within 3 % of the best of a waves x (tiles per
- * range + 8) model, at most 64.  Host-only; returns 1 for invalid sizes.
+ * The number of key ranges streamkl_fwd_splitk uses for splits = 0.  At most 8 query rows
+ * (keys as the MMA's rows, two CTAs per SM): enough ranges for one wave of two CTAs per SM,
+ * 1 when the heads alone fill it.  More rows: 1 when the query blocks alone fill the GPU,
+ * else the fewest ranges within 3 % of the best of a waves x (tiles per range + 8) model, at
+ * most 64.  Uses the current device's SM count.  Host-only; returns 1 for invalid sizes.
  */
 int streamkl_fwd_splits(int B, int Hq, int NQ, int NK);
 
