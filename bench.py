@@ -793,8 +793,10 @@ def run_config(args):
     peak, peak_label, peak_reason = choose_peak(peaks, peak_src, total_s, clk)
     fl = [w.fwd_flops(), w.bwd_flops(), w.bwd_flops()]
     tf = [f / (m * 1e-3) / 1e12 for f, m in zip(fl, ms)]
-    rates = measure_exp_rates(binding, stream, local)
-    exp_roof = exp_roofline(w, ms[0], rates, clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"])
+    exp_roof = None
+    if not args.skip_exp:
+        rates = measure_exp_rates(binding, stream, local)
+        exp_roof = exp_roofline(w, ms[0], rates, clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"])
     line = {
         "metric": "per-workload fwd/bwd ms and TFLOP/s; % of B200 dense bf16 peak",
         "value": sum(fl) / (sum(ms) * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,

@@ -50,3 +50,23 @@ def test_context_usable_after_a_timeout():
     assert np.max(np.abs(gkl - okl) / np.maximum(1, np.abs(okl))) <= KL_TOL
     assert np.max(np.abs(l1.double().cpu().numpy() - ol1)) <= LSE_TOL
     assert np.max(np.abs(l2.double().cpu().numpy() - ol2)) <= LSE_TOL
+
+
+def test_exponential_probe_rates_are_plausible():
+    """The exp2 throughput probe bench.py divides by: both paths run, count their work and
+    land in a plausible band (tens of exp2 per clock per SM at most)."""
+    import torch
+    for kind in (0, 1):
+        rc, n = binding.streamkl_probe_exp2(kind, 200)
+        assert rc == binding.OK and n == 4 * binding.streamkl_num_sms() * 256 * 8 * 200
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        rc, n = binding.streamkl_probe_exp2(kind, 4000)
+        b.record()
+        torch.cuda.synchronize()
+        per_clk_sm = n / (a.elapsed_time(b) * 1e-3) / binding.streamkl_num_sms() / 2.0e9
+        assert 2.0 < per_clk_sm < 64.0, (kind, per_clk_sm)
+    assert binding.streamkl_probe_exp2(2, 10)[0] == binding.ERR_INVALID_ARG
+    assert binding.streamkl_probe_exp2(0, 0)[0] == binding.ERR_INVALID_ARG
+    assert binding.streamkl_device_status() == binding.OK
