@@ -38,6 +38,7 @@ EXPORTS = (
     "streamkl_version",
     "streamkl_probe_exp2",
     "streamkl_num_sms",
+    "streamkl_probe_clock",
 )
 
 _lib = None
@@ -95,6 +96,8 @@ def load(path=None):
     lib.streamkl_probe_exp2.restype = i
     lib.streamkl_num_sms.argtypes = []
     lib.streamkl_num_sms.restype = i
+    lib.streamkl_probe_clock.argtypes = [ctypes.c_longlong, ctypes.c_longlong, vp, i, vp]
+    lib.streamkl_probe_clock.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -196,6 +199,14 @@ def streamkl_probe_exp2(kind, iters, stream=None):
 
 def streamkl_num_sms():
     return load().streamkl_num_sms()
+
+
+def streamkl_probe_clock(duration_ns, interval_ns, samples, stream=None):
+    """Launches the clock probe into `samples` (int64 device tensor of 2 + 2 * max_pairs
+    elements); returns the status."""
+    n = samples.numel()
+    return load().streamkl_probe_clock(int(duration_ns), int(interval_ns), _ptr(samples),
+                                       int((n - 2) // 2), _stream(stream))
 
 
 def status_string(status):

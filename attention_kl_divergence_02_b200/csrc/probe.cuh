@@ -46,4 +46,35 @@ streamkl_probe_exp2_kernel(int iters, int write, float* sink) {
     if (write) sink[blockIdx.x * kProbeThreads + threadIdx.x] = s;
 }
 
+// Effective SM clock.  Under the board's power cap the SM clock drops below its maximum for
+// as long as heavy kernels run, and a sampled clock reading can miss it; clock64 counts the
+// cycles an SM actually runs.  One thread records (globaltimer ns, clock64) pairs every
+// interval_ns for duration_ns, sleeping in between, so that it can share an SM with the
+// kernels being timed (one warp, no shared memory, few registers).  out[0] = pairs written,
+// pair i at out[2 + 2i], out[3 + 2i].  Bounded by the duration and by an iteration cap.
+constexpr long long kClockMaxIters = 1LL << 27;
+
+__global__ void __launch_bounds__(32)
+streamkl_probe_clock_kernel(long long duration_ns, long long interval_ns, int max_pairs,
+                            long long* out) {
+    if (threadIdx.x != 0) return;
+    const long long t0 = (long long)globaltimer();
+    long long next = t0;
+    int n = 0;
+    for (long long it = 0; it < kClockMaxIters && n < max_pairs; ++it) {
+        const long long t = (long long)globaltimer();
+        if (t - t0 > duration_ns) break;
+        if (t >= next) {
+            out[2 + 2 * n] = t;
+            out[3 + 2 * n] = clock64();
+            ++n;
+            next = t + interval_ns;
+        } else {
+            __nanosleep(500);
+        }
+    }
+    out[0] = n;
+    out[1] = 0;
+}
+
 }  // namespace skl

@@ -257,6 +257,20 @@ int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream) {
 
 int streamkl_num_sms(void) { return num_sms(); }
 
+int streamkl_probe_clock(long long duration_ns, long long interval_ns, long long* samples,
+                         int max_pairs, void* stream) {
+    if (!samples) return STREAMKL_ERR_INVALID_ARG;
+    if (duration_ns < 1000 || duration_ns > 10000000000LL || interval_ns < 1000 ||
+        interval_ns > duration_ns || max_pairs < 2)
+        return STREAMKL_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(samples) % 8 != 0) return STREAMKL_ERR_UNSUPPORTED;
+    skl::streamkl_probe_clock_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        duration_ns, interval_ns, max_pairs, samples);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "clock probe launch");
+    return STREAMKL_OK;
+}
+
 }  // extern "C"
 
 namespace {

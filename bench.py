@@ -93,17 +93,22 @@ def choose_peak(peaks, peak_src, timed_s, clk):
     the power cap).  Returns (peak, label, reason)."""
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    med, mx = (clk or {}).get("sm_mhz"), (clk or {}).get("sm_max_mhz")
+    clk = clk or {}
+    mx = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz")
+    eff = clk.get("sm_mhz_effective")
+    med, what = (eff, "effective SM clock (clock probe)") if eff else (
+        clk.get("sm_mhz"), "median sampled SM clock")
     at_max = med is not None and mx is not None and med >= 0.97 * mx
     if timed_s < 1.0 and at_max:
         return burst, "%s bf16_tflops (burst)" % peak_src, (
-            "timed region %.2f s < 1 s and median SM clock %.0f MHz at its maximum %.0f"
-            % (timed_s, med, mx))
+            "timed region %.2f s < 1 s and %s %.0f MHz at its maximum %.0f"
+            % (timed_s, what, med, mx))
     why = []
     if timed_s >= 1.0:
         why.append("timed region %.2f s >= 1 s" % timed_s)
     if not at_max:
-        why.append("median SM clock %s MHz below its maximum %s" % (med, mx))
+        why.append("%s %s MHz below its maximum %s (power cap)" % (
+            what, "%.0f" % med if med is not None else None, mx))
     return sus, "%s bf16_tflops_sustained" % peak_src, "; ".join(why)
 
 
@@ -227,6 +232,51 @@ class ClockSampler:
         med = loaded[len(loaded) // 2] if loaded else None
         return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+class ClockProbe:
+    """Effective SM clock over the timed region, from the library's clock probe: one warp on
+    a stream of its own, beside the timed kernels, records (ns, SM cycles) every 50 us.
+    Under the board's power cap the SM clock drops while the step runs, and the 100 ms
+    nvidia-smi samples can miss it; cycles over nanoseconds cannot."""
+
+    INTERVAL_NS = 50_000
+
+    def __init__(self, binding, device):
+        import torch
+        self.binding, self.torch, self.device = binding, torch, device
+        self.samples = None
+
+    def start(self, expected_ms):
+        torch = self.torch
+        dur_ns = int(min(9.0e9, max(2.0e6, expected_ms * 1.5e6 + 20e6)))
+        pairs = min(400_000, dur_ns // self.INTERVAL_NS + 16)
+        self.samples = torch.zeros(2 + 2 * pairs, dtype=torch.int64, device=self.device)
+        self.stream = torch.cuda.Stream(device=self.device)
+        rc = self.binding.streamkl_probe_clock(dur_ns, self.INTERVAL_NS, self.samples, self.stream)
+        if rc != self.binding.OK:
+            raise RuntimeError("clock probe: %s" % self.binding.status_string(rc))
+
+    def stop(self, region_ms):
+        """Waits for the probe; returns the clock over its first region_ms milliseconds."""
+        self.torch.cuda.synchronize()
+        h = self.samples.cpu().tolist()
+        n = int(h[0])
+        t = [h[2 + 2 * i] for i in range(n)]
+        c = [h[3 + 2 * i] for i in range(n)]
+        if n < 2:
+            return None
+        last = max(i for i in range(n) if t[i] - t[0] <= region_ms * 1e6) if n else 0
+        if last < 1:
+            return None
+        per = sorted((c[i + 1] - c[i]) / (t[i + 1] - t[i]) * 1e3 for i in range(last)
+                     if t[i + 1] > t[i])
+        return {"sm_mhz_effective": (c[last] - c[0]) / (t[last] - t[0]) * 1e3,
+                "sm_mhz_effective_p10": per[len(per) // 10] if per else None,
+                "sm_mhz_effective_p90": per[(9 * len(per)) // 10] if per else None,
+                "pairs": last + 1, "span_ms": (t[last] - t[0]) * 1e-6,
+                "how": "library clock probe beside the timed kernels: SM cycles (clock64) over "
+                       "globaltimer ns every 50 us, first %.1f ms" % region_ms}
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -373,9 +423,14 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
+    wa, wb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        if i == args.warmup - 1:
+            wa.record(stream)
         fwd(); bwd(1); bwd(2)
+    wb.record(stream)
     torch.cuda.synchronize()
+    warm_step_ms = wa.elapsed_time(wb)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
@@ -387,8 +442,10 @@ def run_gpu(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    probe = ClockProbe(binding, dev)
     barrier()
     torch.cuda.synchronize()
+    probe.start(warm_step_ms * args.steps)
     t_start.record(stream)
     for k in range(args.steps):
         ev[k][0].record(stream)
@@ -402,10 +459,14 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    region_ms = t_start.elapsed_time(t_end)
+    eff = probe.stop(region_ms)
+    if eff:
+        clk.update(eff)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = region_ms
     f_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     b1_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     b2_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
@@ -498,7 +559,7 @@ def run_gpu(args):
     exp_roof = None
     if not args.skip_exp:
         rates = measure_exp_rates(binding, stream, local)
-        step_mhz = clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"]
+        step_mhz = clk.get("sm_mhz_effective") or clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"]
         exp_roof = exp_roofline(w, f_ms, rates, step_mhz)
         exp_roof["probe_clocks"] = rates["clocks"]
     line = {
@@ -535,7 +596,7 @@ def run_gpu(args):
                                  "dK convert kernel" if dom.startswith("bwd") else "")},
         "exp_roofline": exp_roof,
         "clocks": clk,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 5 * args.steps + (1 if eff else 0),
         "e2e": e2e,
     }
     if world == 1 and rank == 0 and not args.skip_cpu:
@@ -762,9 +823,14 @@ def run_config(args):
         binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], scale=w.scale,
                     causal=w.causal, out=g, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    wa, wb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        if i == args.warmup - 1:
+            wa.record(stream)
         fwd(); bwd(1); bwd(2)
+    wb.record(stream)
     torch.cuda.synchronize()
+    warm_step_ms = wa.elapsed_time(wb)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
@@ -772,7 +838,9 @@ def run_config(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    probe = ClockProbe(binding, dev)
     torch.cuda.synchronize()
+    probe.start(warm_step_ms * args.steps)
     for k in range(args.steps):
         ev[k][0].record(stream)
         fwd()
@@ -783,6 +851,9 @@ def run_config(args):
         ev[k][3].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
+    eff = probe.stop(ev[0][0].elapsed_time(ev[-1][3]))
+    if eff:
+        clk.update(eff)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
@@ -796,7 +867,8 @@ def run_config(args):
     exp_roof = None
     if not args.skip_exp:
         rates = measure_exp_rates(binding, stream, local)
-        exp_roof = exp_roofline(w, ms[0], rates, clk.get("sm_mhz") or rates["mufu_ex2"]["sm_mhz"])
+        exp_roof = exp_roofline(w, ms[0], rates, clk.get("sm_mhz_effective") or clk.get("sm_mhz")
+                                or rates["mufu_ex2"]["sm_mhz"])
     line = {
         "metric": "per-workload fwd/bwd ms and TFLOP/s; % of B200 dense bf16 peak",
         "value": sum(fl) / (sum(ms) * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
@@ -818,7 +890,7 @@ def run_config(args):
                      "bwd_mode1_frac": tf[1] / peak, "bwd_mode2_frac": tf[2] / peak},
         "exp_roofline": exp_roof,
         "clocks": clk,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 5 * args.steps + (1 if eff else 0),
     }
     if not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline(w, target_s=10.0)

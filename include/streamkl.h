@@ -223,6 +223,26 @@ int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream);
  */
 int streamkl_num_sms(void);
 
+/*
+ * Effective SM clock probe; no part of the KL computation.  Under the board's power cap
+ * the SM clock runs below its maximum while heavy kernels run, so a kernel's time depends
+ * on that clock; this records it while other work runs.  Launches one 32-thread CTA on
+ * `stream` (meant for a stream of its own, concurrent with the work being timed: it needs
+ * no shared memory and sleeps between samples, so it fits beside every kernel of this
+ * library on one SM) whose first thread writes, every `interval_ns`, the pair
+ * (%globaltimer in ns, clock64 of its SM) until `duration_ns` has passed or `max_pairs`
+ * pairs are written.  The effective clock between two pairs is
+ * delta(clock64) / delta(ns) in GHz.
+ *   samples  : device buffer of 2 + 2 * max_pairs int64, 8-byte aligned; on completion
+ *              samples[0] = pairs written, samples[1] = 0, pair i at samples[2 + 2i],
+ *              samples[3 + 2i].
+ *   duration : 1 us to 10 s; interval: 1 us to duration; max_pairs >= 2.
+ * Returns STREAMKL_ERR_INVALID_ARG for an argument outside these ranges (nothing launched),
+ * STREAMKL_ERR_UNSUPPORTED for a misaligned buffer.
+ */
+int streamkl_probe_clock(long long duration_ns, long long interval_ns, long long* samples,
+                         int max_pairs, void* stream);
+
 /* Static text for a status code (never NULL). */
 const char* streamkl_status_string(int status);
 

@@ -163,6 +163,23 @@ def test_splitk_rejects_on_host(lib, kw, want):
     assert splitk_call(_expect=want, **kw) == want
 
 
+@pytest.mark.parametrize("args, want", [
+    ((0, 50_000, 1 << 20, 8), binding.ERR_INVALID_ARG),              # duration below 1 us
+    ((20_000_000_000, 50_000, 1 << 20, 8), binding.ERR_INVALID_ARG),  # above 10 s
+    ((1_000_000, 500, 1 << 20, 8), binding.ERR_INVALID_ARG),          # interval below 1 us
+    ((1_000_000, 2_000_000, 1 << 20, 8), binding.ERR_INVALID_ARG),    # interval above duration
+    ((1_000_000, 50_000, 1 << 20, 1), binding.ERR_INVALID_ARG),       # fewer than 2 pairs
+    ((1_000_000, 50_000, None, 8), binding.ERR_INVALID_ARG),          # no buffer
+    ((1_000_000, 50_000, (1 << 20) + 4, 8), binding.ERR_UNSUPPORTED),  # misaligned buffer
+])
+def test_clock_probe_rejects_on_host(lib, args, want):
+    """The clock probe validates its arguments before launching anything."""
+    dur, iv, ptr, pairs = args
+    assert lib.streamkl_probe_clock(dur, iv, ptr, pairs, None) == want
+    for kind, iters in ((2, 10), (-1, 10), (0, 0)):
+        assert lib.streamkl_probe_exp2(kind, iters, None, None) == binding.ERR_INVALID_ARG
+
+
 def test_header_is_plain_c():
     """The public header compiles as C99 with no CUDA or torch headers."""
     import subprocess

@@ -29,6 +29,17 @@ def test_sustained_peak_otherwise(timed_s, clk):
     assert peak == 1420.9 and "sustained" in label and why
 
 
+def test_effective_clock_decides_over_the_sampled_one():
+    """nvidia-smi may report the maximum clock while the power cap holds the SMs lower; the
+    clock probe's cycles-over-time figure then decides."""
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "sm_mhz_effective": 1725.0}
+    peak, label, why = bench.choose_peak(PEAKS, "measured", 0.25, clk)
+    assert peak == 1420.9 and "sustained" in label and "1725" in why and "power cap" in why
+    clk["sm_mhz_effective"] = 1950.0
+    peak, label, why = bench.choose_peak(PEAKS, "measured", 0.25, clk)
+    assert peak == 1694.5 and "clock probe" in why
+
+
 def test_exp_roofline_of_the_headline_forward():
     w = inputs.WORKLOADS["headline"]
     # 16 ex2 per clock per SM on 148 SMs at 2000 MHz -> 4.736e12 exp2/s; the forward spends 2

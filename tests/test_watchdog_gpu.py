@@ -70,3 +70,36 @@ def test_exponential_probe_rates_are_plausible():
     assert binding.streamkl_probe_exp2(2, 10)[0] == binding.ERR_INVALID_ARG
     assert binding.streamkl_probe_exp2(0, 0)[0] == binding.ERR_INVALID_ARG
     assert binding.streamkl_device_status() == binding.OK
+
+
+def test_clock_probe_reads_a_plausible_clock_beside_a_kernel():
+    """The clock probe, on a stream of its own beside a forward, records monotone time and
+    cycle stamps at about the requested interval and an SM clock between 0.3 and 2.2 GHz;
+    the forward beside it still matches the oracle."""
+    w = inputs.variant(inputs.WORKLOADS["headline"], Hq=2, Hkv=2, NQ=4096, NK=4096)
+    t = inputs.make(w, device="cuda")
+    kl, l1, l2 = (torch.empty((w.B, w.Hq, w.NQ), device="cuda") for _ in range(3))
+    samples = torch.zeros(2 + 2 * 400, dtype=torch.int64, device="cuda")
+    side = torch.cuda.Stream()
+    assert binding.streamkl_probe_clock(20_000_000, 100_000, samples, side) == binding.OK
+    for _ in range(5):
+        binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=True, out=(kl, l1, l2))
+    torch.cuda.synchronize()
+    h = samples.cpu().tolist()
+    n = h[0]
+    assert 100 <= n <= 400, n
+    ts = [h[2 + 2 * i] for i in range(n)]
+    cs = [h[3 + 2 * i] for i in range(n)]
+    assert all(b > a for a, b in zip(ts, ts[1:])) and all(b > a for a, b in zip(cs, cs[1:]))
+    assert 19e6 <= ts[-1] - ts[0] <= 21e6
+    gaps = sorted(b - a for a, b in zip(ts, ts[1:]))
+    assert 90_000 <= gaps[len(gaps) // 2] <= 150_000
+    mhz = (cs[-1] - cs[0]) / (ts[-1] - ts[0]) * 1e3
+    assert 300 < mhz < 2200, mhz
+    assert binding.streamkl_device_status() == binding.OK
+    rows = np.arange(0, w.B * w.Hq * w.NQ, 97)
+    okl, ol1, _ = oracle.fwd_rows(*[inputs.to_f64(t[k]) for k in ("q1", "k1", "q2", "k2")], rows,
+                                  scale=w.scale, causal=True)
+    gkl = kl.double().cpu().numpy().reshape(-1)[rows]
+    assert np.max(np.abs(gkl - okl) / np.maximum(1, np.abs(okl))) <= KL_TOL
+    assert np.max(np.abs(l1.double().cpu().numpy().reshape(-1)[rows] - ol1)) <= LSE_TOL
