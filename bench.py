@@ -723,10 +723,15 @@ def run_chunk(args):
         binding.bwd(mode, t["q1"], t["k1"], t["q2"], t["k2"], kl, l1, l2, t["dkl"], scale=w.scale,
                     out=g, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    wa, wb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        if i == args.warmup - 1:
+            wa.record(stream)
         bwd(1)
         bwd(2)
+    wb.record(stream)
     torch.cuda.synchronize()
+    warm_ms = wa.elapsed_time(wb)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after warm-up: %s" % binding.status_string(st))
@@ -745,16 +750,27 @@ def run_chunk(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    probe = ClockProbe(binding, dev)
+    torch.cuda.synchronize()
+    probe.start(warm_ms * args.steps)
+    r0 = torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
     m1 = timed(1)
     m2 = timed(2)
+    r1 = torch.cuda.Event(enable_timing=True)
+    r1.record(stream)
     clk = clocks.stop()
+    eff = probe.stop(r0.elapsed_time(r1))
+    if eff:
+        clk.update(eff)
     st = binding.streamkl_device_status()
     if st != binding.OK:
         raise RuntimeError("device status after the timed region: %s" % binding.status_string(st))
     flops = w.bwd_flops()
     t1, t2 = flops / (m1 * 1e-3) / 1e12, flops / (m2 * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_label, peak_reason = choose_peak(peaks, peak_src, (m1 + m2) * args.steps * 1e-3, clk)
     line = {
         "metric": "backward TFLOP/s, query chunk against a long context (key-range backward)",
         "value": 2 * flops / ((m1 + m2) * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
@@ -768,11 +784,12 @@ def run_chunk(args):
         "bwd_mode1_ms": m1, "bwd_mode1_tflops": t1, "bwd_mode2_ms": m2, "bwd_mode2_tflops": t2,
         "roofline": {"bound": "tensor", "kernel": "bwd_mode1", "achieved": t1, "peak": peak,
                      "unit": "TFLOP/s", "frac": t1 / peak, "traffic": None,
-                     "peak_source": "%s bf16_tflops (burst)" % peak_src,
+                     "bwd_mode2_frac": t2 / peak, "frac_of_burst": t1 / burst,
+                     "peak_source": peak_label, "peak_rule": peak_reason,
                      "note": "achieved = algorithmic FLOPs (8d per pair) / CUDA-event time of the "
                              "call (memset, kernel, dK and dQ converts)"},
         "clocks": clk,
-        "gpu_launches": 3 * 2 * args.steps,
+        "gpu_launches": 3 * 2 * args.steps + (1 if eff else 0),
     }
     print(json.dumps(line), flush=True)
     return 0
