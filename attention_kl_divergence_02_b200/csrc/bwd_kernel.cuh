@@ -73,16 +73,22 @@ constexpr int kBwdProducerWarp = 20;
 constexpr int kBwdMmaWarp = 21;
 constexpr int kBwdHeadGroup = 2;   // (batch, head) planes scheduled together
 
-template <int D, bool SHARED_K>
+// HP = query heads per CTA (1, or 2 at d = 64 when a KV group has an even number of query
+// heads: the CTA then owns the same query tile of two heads that share their keys, visits
+// every key tile once per head, and the dK partial of a key tile sums both heads' visits in
+// TMEM before it is reduced).
+template <int D, bool SHARED_K, int HP = 1>
 struct BwdCfg {
+    static_assert(HP == 1 || (HP == 2 && D == 64), "two heads per CTA only at d = 64");
     static constexpr int kTile = 128 * D * 2;                      // one 128-row bf16 tile
     static constexpr int kBoxes = D / 64;
     static constexpr int kBox = 128 * 128;
-    static constexpr int kPerVisit = SHARED_K ? 1 : 2;             // key tiles streamed per visit
-    static constexpr int kSlots = (D == 128) ? 3 : 8;              // key-tile ring
-    static constexpr int kQ1 = 0;
+    static constexpr int kPerVisit = SHARED_K ? 1 : 2;             // key tiles streamed per key step
+    static constexpr int kSlots = (D == 128) ? 3 : (HP == 2 ? 6 : 8);   // key-tile ring
+    static constexpr int kQ1 = 0;                                  // head slot hs: + hs*kQStride
     static constexpr int kQ2 = kTile;
-    static constexpr int kRing = 2 * kTile;                        // slot s at kRing + s*kTile
+    static constexpr int kQStride = 2 * kTile;
+    static constexpr int kRing = HP * 2 * kTile;                   // slot s at kRing + s*kTile
     static constexpr int kDS = kRing + kSlots * kTile;             // dS tiles, 2 x 128 x 128 bf16
     static constexpr int kDSBuf = 128 * 128 * 2;                   // dS tile b at kDS + b*kDSBuf
     static constexpr int kBar = kDS + 2 * kDSBuf;
@@ -101,6 +107,7 @@ struct BwdCfg {
     static constexpr int kNumBars = DONE + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kSmem = kMisc + 16 + 1024;
+    // dQ of head slot hs at kColDQ + hs*D (HP = 2 only at d = 64: columns 256..383)
     static constexpr uint32_t kColS1 = 0, kColS2 = 128, kColDQ = 256, kColDK = 384;
 };
 
@@ -203,12 +210,12 @@ __device__ __forceinline__ void ds_chunk_any(bool masked, bool folded, const uin
     }
 }
 
-template <int D, bool SHARED_K, int MODE>
+template <int D, bool SHARED_K, int MODE, int HP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK1, const __grid_constant__ CUtensorMap tmK2,
                     const BwdParams p) {
-    using C = BwdCfg<D, SHARED_K>;
+    using C = BwdCfg<D, SHARED_K, HP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -227,8 +234,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     // the partial sums meet in L2 instead of going back and forth to DRAM (a group of 2
     // measured best of 2, 4, 8 and 16 on the causal and GQA workloads).
     // With key ranges (few query tiles, many keys), the ranges of one query tile are
-    // neighbours in the grid.
-    const int BH = p.B * p.Hq;
+    // neighbours in the grid.  With HP = 2 a "plane" is a pair of query heads (h, h+1) of one
+    // KV group.
+    const int HU = p.Hq / HP;                 // head units per batch
+    const int BH = p.B * HU;
     const int sp = blockIdx.x % p.splits;
     const int ub = blockIdx.x / p.splits;
     const int per_group = kBwdHeadGroup * p.nqt;
@@ -236,14 +245,16 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     const int gh = min(kBwdHeadGroup, BH - group * kBwdHeadGroup);   // planes in this group
     const int r_in = ub - group * per_group;
     const int unit = r_in / gh;
-    const int bh = group * kBwdHeadGroup + r_in % gh;
+    const int bhu = group * kBwdHeadGroup + r_in % gh;
     const int qt = p.causal ? (p.nqt - 1 - unit) : unit;
-    const int b = bh / p.Hq;
-    const int h = bh % p.Hq;
+    const int b = bhu / HU;
+    const int h = (bhu % HU) * HP;            // first query head of the unit
+    const int bh = b * p.Hq + h;              // its (batch, head) plane; head slot hs is bh + hs
     const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
     const int q0 = qt * 128;
     const BwdSchedule sched(p, qt, h, sp);
-    const int N = sched.count;
+    const int N = sched.count;                // key steps; visit v = key step v / HP, head slot v % HP
+    const int V = N * HP;
     constexpr bool mode1 = (MODE == 1);
     // Key tiles of a visit enter the ring in the order (fixed distribution's, free
     // distribution's): j = 0 is released as soon as S is done, j = 1 after dQ.  With three
@@ -254,7 +265,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
     constexpr int kJ1 = SHARED_K ? 0 : (mode1 ? 0 : 1);
     constexpr int kJ2 = SHARED_K ? 0 : (mode1 ? 1 : 0);
     constexpr int kJFree = SHARED_K ? 0 : 1;
-    const uint32_t qfree = sb + (mode1 ? C::kQ2 : C::kQ1);
+    const uint32_t qfree = sb + (mode1 ? C::kQ2 : C::kQ1);   // head slot hs: + hs*kQStride
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(C::Q_FULL), 1);
@@ -264,8 +275,10 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         }
         mbar_init(BAR(C::S_FULL), 1);
         mbar_init(BAR(C::S_FREE), 32 * 4 * kBwdWG);
+        // the flush warps' "dK read out" arrival gates the visits that start a key step's dK:
+        // every visit when HP = 1, the even ones (tile 0) when HP = 2
         for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(C::DS_FULL + b), 32 * 4 * kBwdWG + 128);
+            mbar_init(BAR(C::DS_FULL + b), 32 * 4 * kBwdWG + ((HP == 1 || b == 0) ? 128 : 0));
             mbar_init(BAR(C::DS_FREE + b), 1);
         }
         mbar_init(BAR(C::DK_FULL), 1);
@@ -290,11 +303,14 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             tma_prefetch_desc(&tmQ2);
             tma_prefetch_desc(&tmK1);
             if (!SHARED_K) tma_prefetch_desc(&tmK2);
-            mbar_arrive_expect_tx(BAR(C::Q_FULL), 2 * C::kTile);
-            for (int bx = 0; bx < C::kBoxes; ++bx) {
-                tma_load_3d(sb + C::kQ1 + bx * C::kBox, &tmQ1, BAR(C::Q_FULL), bx * 64, q0, bh);
-                tma_load_3d(sb + C::kQ2 + bx * C::kBox, &tmQ2, BAR(C::Q_FULL), bx * 64, q0, bh);
-            }
+            mbar_arrive_expect_tx(BAR(C::Q_FULL), HP * 2 * C::kTile);
+            for (int hs = 0; hs < HP; ++hs)
+                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                    tma_load_3d(sb + C::kQ1 + hs * C::kQStride + bx * C::kBox, &tmQ1, BAR(C::Q_FULL),
+                                bx * 64, q0, bh + hs);
+                    tma_load_3d(sb + C::kQ2 + hs * C::kQStride + bx * C::kBox, &tmQ2, BAR(C::Q_FULL),
+                                bx * 64, q0, bh + hs);
+                }
             uint32_t it = 0;
             bool ok = true;
             for (int n = 0; n < N && ok; ++n) {
@@ -341,8 +357,11 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             const uint64_t dq1k = sw128_desc(sb + C::kQ1, 16, 1024);        // Q1, K-major
             const uint64_t dq2k = sw128_desc(sb + C::kQ2, 16, 1024);        // Q2, K-major
             const uint64_t dqfm = sw128_desc(qfree, C::kBox, 1024);         // Q_free, MN-major
-            // S of visit n; returns false if a wait gave up
-            auto issue_S = [&](int n) -> bool {
+            constexpr uint32_t kQS = (uint32_t)C::kQStride;                  // next head slot's Q
+            // S of visit v (key step v / HP, head slot v % HP); returns false if a wait gave up
+            auto issue_S = [&](int v) -> bool {
+                const int n = v / HP;
+                const uint32_t qo = (uint32_t)(v % HP) * kQS;
                 const uint32_t s1 = slot_of(n, kJ1);
                 const uint32_t s2 = SHARED_K ? s1 : slot_of(n, kJ2);
                 if (!mbar_wait(BAR(C::K_FULL + s1), fill_parity(n, kJ1), abort_flag)) return false;
@@ -354,48 +373,55 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS1, dadd(dq1k, off), dadd(dk1, off), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS1, dadd(dq1k, qo + off), dadd(dk1, off), idS, k > 0);
                 }
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * C::kBox + (k & 3) * 32;
-                    mma_bf16_ss(tmem + C::kColS2, dadd(dq2k, off), dadd(dk2, off), idS, k > 0);
+                    mma_bf16_ss(tmem + C::kColS2, dadd(dq2k, qo + off), dadd(dk2, off), idS, k > 0);
                 }
                 mma_commit(BAR(C::S_FULL));
-                // with distinct keys, the fixed distribution's key tile (j = 0) is done after S
-                if (!SHARED_K) mma_commit(BAR(C::K_EMPTY + slot_of(n, 0)));
+                // with distinct keys, the fixed distribution's key tile (j = 0) is done after the
+                // key step's last S
+                if (!SHARED_K && v % HP == HP - 1) mma_commit(BAR(C::K_EMPTY + slot_of(n, 0)));
                 return true;
             };
-            // dQ of visit m, once its dS tile is written (and the flush has read dK of m-1)
+            // dQ of visit m, once its dS tile is written (and the flush has read the dK of the
+            // previous key step, when m starts one)
             auto issue_dq = [&](int m) -> bool {
+                const int n = m / HP;
+                const int hs = m % HP;
                 const uint32_t ds = sb + C::kDS + (m & 1) * C::kDSBuf;
                 const uint64_t ddsk = sw128_desc(ds, 16, 1024);         // dS, K-major (A of dQ)
-                const uint64_t dkfm = sw128_desc(sb + C::kRing + slot_of(m, kJFree) * C::kTile,
+                const uint64_t dkfm = sw128_desc(sb + C::kRing + slot_of(n, kJFree) * C::kTile,
                                                  C::kBox, 1024);        // K_free, MN-major
                 if (!mbar_wait(BAR(C::DS_FULL + (m & 1)), (m >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                // dQ += dS K_free, accumulated over every visit
+                // dQ of head slot hs += dS K_free, accumulated over every visit of that slot
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 keys, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDQ, dadd(ddsk, (k >> 2) * C::kBox + (k & 3) * 32),
-                                dadd(dkfm, k * 2048), idQ, (m > 0 || k > 0));
+                    mma_bf16_ss(tmem + C::kColDQ + (uint32_t)(hs * D),
+                                dadd(ddsk, (k >> 2) * C::kBox + (k & 3) * 32),
+                                dadd(dkfm, k * 2048), idQ, (m >= HP || k > 0));
                 }
-                mma_commit(BAR(C::K_EMPTY + slot_of(m, kJFree)));
+                if (hs == HP - 1) mma_commit(BAR(C::K_EMPTY + slot_of(n, kJFree)));
                 return true;
             };
-            // dK partial of visit m: dS^T Q_free (fresh every visit); frees its dS tile
+            // dK partial of visit m: dS^T Q_free of its head slot, fresh at a key step's first
+            // visit and accumulated over the others; frees its dS tile
             auto issue_dk = [&](int m) {
+                const int hs = m % HP;
                 const uint64_t ddsm = sw128_desc(sb + C::kDS + (m & 1) * C::kDSBuf, C::kBox, 1024);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {   // 128 queries, 16 per MMA
-                    mma_bf16_ss(tmem + C::kColDK, dadd(ddsm, k * 2048), dadd(dqfm, k * 2048), idK,
-                                k > 0);
+                    mma_bf16_ss(tmem + C::kColDK, dadd(ddsm, k * 2048),
+                                dadd(dqfm, (uint32_t)hs * kQS + k * 2048), idK, (hs > 0 || k > 0));
                 }
-                mma_commit(BAR(C::DK_FULL));
+                if (hs == HP - 1) mma_commit(BAR(C::DK_FULL));
                 mma_commit(BAR(C::DS_FREE + (m & 1)));
             };
             bool ok = mbar_wait(BAR(C::Q_FULL), 0, abort_flag);
-            if (ok && N > 0) ok = issue_S(0);
+            if (ok && V > 0) ok = issue_S(0);
             if constexpr (D == 64) {
             // Issue order dQ(n-1), S(n+1), dK(n-1): the tensor core executes in issue order, so
             // S(n+1) -- which the compute warps wait for -- queues behind 8 dQ MMAs instead of
@@ -403,24 +429,24 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
             // two dS tiles cover the later dK.  Measured faster at d = 64 (GQA, mode 1: 6.83 ->
             // 6.4 ms), slower at d = 128 (headline 4.33 -> 4.8 ms), so d = 128 keeps the order
             // S(n+1), dQ(n), dK(n).
-            for (int n = 0; n <= N && ok; ++n) {
-                if (n >= 1 && !issue_dq(n - 1)) break;
-                if (n + 1 < N) {
-                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+            for (int v = 0; v <= V && ok; ++v) {
+                if (v >= 1 && !issue_dq(v - 1)) break;
+                if (v + 1 < V) {
+                    if (!mbar_wait(BAR(C::S_FREE), v & 1, abort_flag)) break;
                     tc_fence_after();
-                    if (!issue_S(n + 1)) break;
+                    if (!issue_S(v + 1)) break;
                 }
-                if (n >= 1) issue_dk(n - 1);
+                if (v >= 1) issue_dk(v - 1);
             }
             } else {
-            for (int n = 0; n < N && ok; ++n) {
-                if (n + 1 < N) {
-                    if (!mbar_wait(BAR(C::S_FREE), n & 1, abort_flag)) break;
+            for (int v = 0; v < V && ok; ++v) {
+                if (v + 1 < V) {
+                    if (!mbar_wait(BAR(C::S_FREE), v & 1, abort_flag)) break;
                     tc_fence_after();
-                    if (!issue_S(n + 1)) break;
+                    if (!issue_S(v + 1)) break;
                 }
-                if (!issue_dq(n)) break;
-                issue_dk(n);
+                if (!issue_dq(v)) break;
+                issue_dk(v);
             }
             }
             mma_commit(BAR(C::DQ_DONE));
@@ -432,7 +458,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         const int quarter = warp;               // TMEM lanes 32*quarter.. = key rows
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         mbar_arrive(BAR(C::DS_FULL));               // visit 0 has no earlier dK to wait for
-        for (int n = 0; n < N; ++n) {
+        for (int n = 0; n < N; ++n) {               // one dK partial per key step
             const int kt = sched.key_tile(n);
             if (!mbar_wait(BAR(C::DK_FULL), n & 1, abort_flag)) break;
             tc_fence_after();
@@ -445,9 +471,9 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 tmem_ld32(lane_base + C::kColDK + c * 32, v[0]);
                 tmem_ld32(lane_base + C::kColDK + c * 32 + 32, v[1]);
                 tmem_wait_ld();
-                if (c + 2 == D / 32) {           // the dK columns are all in registers:
-                    tc_fence_before();           // visit n+1 may overwrite them
-                    mbar_arrive(BAR(C::DS_FULL + ((n + 1) & 1)));
+                if (c + 2 == D / 32) {           // the dK columns are all in registers: the
+                    tc_fence_before();           // next key step's first visit may overwrite them
+                    mbar_arrive(BAR(C::DS_FULL + (((n + 1) * HP) & 1)));
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
@@ -469,30 +495,46 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
         // this thread's 64 bytes of dS row r in tile 0: box (wg/2), 16-byte chunks 4*(wg&1)..+3
         uint8_t* ds_row0 = smem + C::kDS + (wg >> 1) * C::kBox + r * 128;
         const int q = q0 + r;
-        // this row's statistics, for the CTA's whole life: a = LSE1*log2(e), bq = LSE2*log2(e)
-        // (mode 1) or LSE2 - LSE1 - KL (mode 2), g; rows past NQ get g = 0 (their dS is 0)
-        float a = 0.f, bq = 0.f, g = 0.f;
-        if (q < p.NQ) {
-            const size_t o = (size_t)bh * p.NQ + q;
-            const float L1 = p.lse1[o], L2 = p.lse2[o];
-            a = L1 * LOG2E;
-            bq = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
-            g = p.dkl[o];
-        }
-        // fold g into the exponents when no row of the warp has g < 0
-        const bool folded = !__any_sync(0xffffffffu, g < 0.f);
-        if (folded && g > 0.f) {
-            const float lg = log2f(g);
-            a -= lg;
-            if (mode1) bq -= lg;
-        }
+        // this row's statistics in each head slot, for the CTA's whole life: a = LSE1*log2(e),
+        // bq = LSE2*log2(e) (mode 1) or LSE2 - LSE1 - KL (mode 2), g; rows past NQ get g = 0
+        // (their dS is 0).  g is folded into the exponents when no row of the warp has g < 0;
         // a row with g = 0 (or past NQ) has dS = 0 exactly: it takes the masked variant with
         // every column masked (folding log2 0 = -inf would leave 2^-126 where the FMA-pipe
         // exponential clamps its argument)
-        const bool zero_row = !(g != 0.f);
+        float a_[HP], bq_[HP], g_[HP];
+        bool folded_[HP], zero_[HP];
+#pragma unroll
+        for (int hs = 0; hs < HP; ++hs) {
+            float a = 0.f, bq = 0.f, g = 0.f;
+            if (q < p.NQ) {
+                const size_t o = (size_t)(bh + hs) * p.NQ + q;
+                const float L1 = p.lse1[o], L2 = p.lse2[o];
+                a = L1 * LOG2E;
+                bq = mode1 ? L2 * LOG2E : (L2 - L1 - p.kl[o]);
+                g = p.dkl[o];
+            }
+            const bool folded = !__any_sync(0xffffffffu, g < 0.f);
+            if (folded && g > 0.f) {
+                const float lg = log2f(g);
+                a -= lg;
+                if (mode1) bq -= lg;
+            }
+            a_[hs] = a;
+            bq_[hs] = bq;
+            g_[hs] = g;
+            folded_[hs] = folded;
+            zero_[hs] = !(g != 0.f);
+        }
         const int kc0 = wg * 32;
         bool ok = true;
-        for (int n = 0; n < N; ++n) {
+        for (int v = 0; v < V; ++v) {
+            const int n = v / HP;
+            const bool h1 = HP == 2 && (v & 1);   // head slot 1 (constant-index selects)
+            const float a = h1 ? a_[HP - 1] : a_[0];
+            const float bq = h1 ? bq_[HP - 1] : bq_[0];
+            const float g = h1 ? g_[HP - 1] : g_[0];
+            const bool folded = h1 ? folded_[HP - 1] : folded_[0];
+            const bool zero_row = h1 ? zero_[HP - 1] : zero_[0];
             const int kt = sched.key_tile(n);
             const int k0 = kt * 128;
             // masked columns: keys past the diagonal of a causal diagonal tile, and
@@ -507,7 +549,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                 need_mask = true;
                 lim = 0;
             }
-            if (!mbar_wait(BAR(C::S_FULL), n & 1, abort_flag)) {
+            if (!mbar_wait(BAR(C::S_FULL), v & 1, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -533,12 +575,12 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     mbar_arrive(BAR(C::S_FREE));  // all of this thread's S columns are read
                 }
             }
-            // dS tile n&1 was last read by the MMAs of visit n-2
-            if (n > 1 && !mbar_wait(BAR(C::DS_FREE + (n & 1)), ((n >> 1) - 1) & 1, abort_flag)) {
+            // dS tile v&1 was last read by the MMAs of visit v-2
+            if (v > 1 && !mbar_wait(BAR(C::DS_FREE + (v & 1)), ((v >> 1) - 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
-            uint8_t* ds_row = ds_row0 + (n & 1) * C::kDSBuf;
+            uint8_t* ds_row = ds_row0 + (v & 1) * C::kDSBuf;
             const int cbase = (wg & 1) * 4;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -547,24 +589,26 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
             }
             fence_async_smem();
-            mbar_arrive(BAR(C::DS_FULL + (n & 1)));
+            mbar_arrive(BAR(C::DS_FULL + (v & 1)));
         }
         // dQ of this query tile, accumulated over every visit of the CTA.  One key range:
         // scale, round, store.  Several: add it into the fp32 dQ workspace (the convert kernel
         // scales and rounds once every range has added its part).
         if (ok && N > 0 && mbar_wait(BAR(C::DQ_DONE), 0, abort_flag)) {
             tc_fence_after();
+#pragma unroll 1
+            for (int hs = 0; hs < HP; ++hs) {
             constexpr int kCols = D / 4;          // dQ columns per warpgroup
             uint32_t v[kCols];
             if constexpr (D == 128) {
                 tmem_ld32(lane_base + C::kColDQ + wg * kCols, v);
             } else {
-                tmem_ld16(lane_base + C::kColDQ + wg * kCols, v);
+                tmem_ld16(lane_base + C::kColDQ + hs * D + wg * kCols, v);
             }
             tmem_wait_ld();
             if (p.splits > 1) {
                 // tile-blocked: [quarter][32-column chunk][4-column group][lane][4]
-                float* blk = p.dq_ws + ((size_t)bh * p.nqt + qt) * (128 * D) +
+                float* blk = p.dq_ws + ((size_t)(bh + hs) * p.nqt + qt) * (128 * D) +
                              (size_t)quarter * (32 * D) + lane * 4;
                 const int c = (wg * kCols) / 32;          // chunk of this warpgroup's columns
                 const int g0 = ((wg * kCols) % 32) / 4;   // first 4-column group in the chunk
@@ -573,7 +617,8 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     red_add_v4(blk + c * 1024 + (g0 + g) * 128, v[4 * g], v[4 * g + 1], v[4 * g + 2],
                                v[4 * g + 3]);
             } else if (q < p.NQ) {
-                uint4* dst = reinterpret_cast<uint4*>(p.dq + ((size_t)bh * p.NQ + q) * D + wg * kCols);
+                uint4* dst = reinterpret_cast<uint4*>(p.dq + ((size_t)(bh + hs) * p.NQ + q) * D +
+                                                      wg * kCols);
 #pragma unroll
                 for (int k = 0; k < kCols / 8; ++k) {
                     float f[8];
@@ -582,6 +627,7 @@ streamkl_bwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
                     dst[k] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]),
                                         pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
                 }
+            }
             }
         }
     }

@@ -165,12 +165,13 @@ int launch_convert(const float* ws, uint16_t* out, int planes, int rows, int nti
     return STREAMKL_OK;
 }
 
-template <int D, bool SHARED>
+template <int D, bool SHARED, int HP>
 int launch_bwd(int mode, const CUtensorMap& q1, const CUtensorMap& q2, const CUtensorMap& k1,
                const CUtensorMap& k2, const skl::BwdParams& p, int grid, size_t ws_bytes,
                uint16_t* dk, cudaStream_t st) {
-    auto kern = mode == 1 ? skl::streamkl_bwd_kernel<D, SHARED, 1> : skl::streamkl_bwd_kernel<D, SHARED, 2>;
-    constexpr int smem = skl::BwdCfg<D, SHARED>::kSmem;
+    auto kern = mode == 1 ? skl::streamkl_bwd_kernel<D, SHARED, 1, HP>
+                          : skl::streamkl_bwd_kernel<D, SHARED, 2, HP>;
+    constexpr int smem = skl::BwdCfg<D, SHARED, HP>::kSmem;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     cudaError_t e = cudaMemsetAsync(p.dk_ws, 0, ws_bytes, st);
@@ -464,11 +465,18 @@ int streamkl_fwd_splitk(const uint16_t* q1, const uint16_t* k1, const uint16_t* 
 
 namespace {
 
+// Query heads per backward CTA: 2 at d = 64 when every KV group has an even number of query
+// heads (the two heads' dK partials of a key tile then meet in tensor memory and their key
+// tiles are loaded once), else 1.  At d = 128 tensor memory has no room for a second dQ.
+int bwd_heads_per_cta(int Hq, int Hkv, int d) {
+    return (d == 64 && (Hq / Hkv) % 2 == 0) ? 2 : 1;
+}
+
 // Key ranges per query tile for the backward: 1 when the query tiles fill the GPU, else the
 // fewest ranges within 3 % of the best of a waves x (tiles per range + 6) model (6 tiles of
 // fixed cost per CTA: query load, pipeline fill, dQ reduction), at most 32.
-int bwd_splits(int B, int Hq, int NQ, int NK) {
-    const long long ctas = (long long)B * Hq * ((NQ + 127) / 128);
+int bwd_splits(int B, int Hq, int Hkv, int NQ, int NK, int d) {
+    const long long ctas = (long long)B * (Hq / bwd_heads_per_cta(Hq, Hkv, d)) * ((NQ + 127) / 128);
     const int nkt = (NK + 127) / 128;
     const int sms = num_sms();
     if (ctas >= sms || nkt < 2) return 1;
@@ -503,7 +511,7 @@ extern "C" {
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d) {
     if (B < 1 || Hq < 1 || Hkv < 1 || NQ < 1 || NK < 1 || (d != 64 && d != 128)) return 0;
     size_t bytes = bwd_dk_bytes(B, Hkv, NK, d);
-    if (bwd_splits(B, Hq, NQ, NK) > 1)   // plus the dQ partial sums, tile-blocked
+    if (bwd_splits(B, Hq, Hkv, NQ, NK, d) > 1)   // plus the dQ partial sums, tile-blocked
         bytes += (size_t)B * Hq * ((NQ + 127) / 128 * 128) * d * sizeof(float);
     return bytes;
 }
@@ -538,23 +546,27 @@ int streamkl_bwd(int mode, const uint16_t* q1, const uint16_t* k1, const uint16_
     p.kl = kl; p.lse1 = lse1; p.lse2 = lse2; p.dkl = dkl;
     p.dk_ws = static_cast<float*>(workspace);
     p.dq = dq;
-    p.splits = bwd_splits(B, Hq, NQ, NK);
+    p.splits = bwd_splits(B, Hq, Hkv, NQ, NK, d);
+    const int hp = bwd_heads_per_cta(Hq, Hkv, d);
     {
         int used;
         split_ranges(NK, p.splits, &p.kps, &used);
         p.splits = used;
     }
     p.dq_ws = p.splits > 1 ? p.dk_ws + bwd_dk_bytes(B, Hkv, NK, d) / sizeof(float) : nullptr;
-    const long long grid = (long long)B * Hq * p.nqt * p.splits;
+    const long long grid = (long long)B * (Hq / hp) * p.nqt * p.splits;
     if (grid >= (1ll << 31)) return STREAMKL_ERR_UNSUPPORTED;
     const size_t ws = streamkl_bwd_workspace_bytes(B, Hq, Hkv, NQ, NK, d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 128) {
-        return shared ? launch_bwd<128, true>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
-                      : launch_bwd<128, false>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
+        return shared ? launch_bwd<128, true, 1>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
+                      : launch_bwd<128, false, 1>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
     }
-    return shared ? launch_bwd<64, true>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
-                  : launch_bwd<64, false>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
+    if (hp == 2)
+        return shared ? launch_bwd<64, true, 2>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
+                      : launch_bwd<64, false, 2>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
+    return shared ? launch_bwd<64, true, 1>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st)
+                  : launch_bwd<64, false, 1>(mode, mq1, mq2, mk1, mk2, p, (int)grid, ws, dk, st);
 }
 
 }  // extern "C"
