@@ -535,14 +535,19 @@ def run_gpu(args):
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        e_probe = ClockProbe(binding, dev)
+        e_probe.start(ms_step * ne * 1.2)
         a.record(stream)
         e2e_run(ne)
         stream.wait_stream(copy_stream)
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks([a.elapsed_time(b) / ne], device=dev)[0]
+        e_region = a.elapsed_time(b)
+        e_eff = e_probe.stop(e_region)
+        e_ms = max_over_ranks([e_region / ne], device=dev)[0]
         e2e = {"value": job_tflops(world, step_flops, e_ms), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "sm_mhz_effective": e_eff["sm_mhz_effective"] if e_eff else None,
                "note": "public API with pinned host buffers; each step copies its own inputs in "
                        "(overlapped with the previous step's compute on a second stream) and "
                        "reads its result (KL, LSE1, LSE2) back"}

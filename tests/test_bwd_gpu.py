@@ -48,6 +48,11 @@ CASES = [
     (1, 1, 1, 1, 1, 128, False, True),
     (1, 1, 1, 40, 40, 128, True, True),
     (1, 2, 1, 3, 700, 128, False, False),
+    # d = 64 with an even KV-group size: two query heads per CTA (their dK partials summed on
+    # chip); causal with a ragged last tile, 4:1 shared keys, and two KV groups with B = 2
+    (1, 4, 2, 333, 333, 64, True, False),
+    (1, 8, 2, 257, 257, 64, True, True),
+    (2, 4, 2, 130, 1000, 64, False, False),
 ]
 
 

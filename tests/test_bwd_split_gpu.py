@@ -32,6 +32,8 @@ CASES = [
     (1, 2, 1, 64, 5000, 128, False, True),      # GQA, ragged keys
     (1, 1, 1, 640, 640, 128, True, True),       # causal: late ranges of early tiles are empty
     (2, 2, 2, 130, 1900, 64, False, False),
+    (1, 4, 2, 200, 4000, 64, False, False),     # two query heads per CTA, key ranges
+    (1, 4, 2, 384, 384, 64, True, True),        # the same, causal
 ]
 
 
