@@ -59,6 +59,38 @@ def test_peaked_and_flat_rows():
     check_fwd(got, want, "peaked")
 
 
+def test_score_jumps_above_the_running_maximum():
+    """Rows whose scores jump far above the maximum of the keys before them, in a later key
+    tile, so the online rescale must carry the earlier sums down by that much: row 0 jumps by
+    ~131 binary orders (2^-131 underflows fp32 -- the earlier keys must drop out, not turn
+    into NaN), row 1 by ~78, row 2 by ~49; the other rows see moderate scores from the same
+    keys.  Both distributions against the oracle, shared keys and distinct ones."""
+    for shared in (True, False):
+        w = inputs.custom(1, 1, 1, 256, 1024, 128, False, shared, seed=21)
+        t = inputs.make(w, device="cpu")
+        q1 = t["q1"].float()
+        keys = {"k1": t["k1"].float() * 0.1}
+        if not shared:
+            keys["k2"] = t["k2"].float() * 0.1
+        for key, row, c in ((700, 0, 8.0), (900, 1, 4.8), (950, 2, 3.0)):
+            # a key along the row's query, scaled so that scale * <q1, k> = c * 128 * scale
+            # nats = 16.3 * c binary orders above the earlier keys' near-zero scores
+            qr = q1[0, 0, row]
+            for name in keys:
+                keys[name][0, 0, key] = c * 128.0 * qr / float(qr @ qr)
+        t["k1"] = keys["k1"].to(torch.bfloat16)
+        t["k2"] = t["k1"] if shared else keys["k2"].to(torch.bfloat16)
+        t = {k: v.cuda() for k, v in t.items()}
+        if shared:
+            t["k2"] = t["k1"]
+        got = run_fwd(t, w)
+        want = oracle.fwd(host64(t["q1"]), host64(t["k1"]), host64(t["q2"]), host64(t["k2"]),
+                          scale=w.scale, causal=False)
+        check_fwd(got, want, "score jumps, shared=%s" % shared)
+        # the jumps are as large as intended: LSE1 of rows 0-2 far above the others
+        assert got[1][0, 0, 0] > 80 and got[1][0, 0, 1] > 45 and got[1][0, 0, 2] > 28
+
+
 def test_identical_inputs_give_zero_kl():
     w = inputs.custom(1, 2, 2, 300, 300, 128, True, True, seed=3)
     t = inputs.make(w, device="cuda")
