@@ -204,6 +204,10 @@ def streamkl_num_sms():
 def streamkl_probe_clock(duration_ns, interval_ns, samples, stream=None):
     """Launches the clock probe into `samples` (int64 device tensor of 2 + 2 * max_pairs
     elements); returns the status."""
+    import torch
+    if samples.dtype != torch.int64 or not samples.is_cuda or not samples.is_contiguous() \
+            or samples.numel() < 6:
+        raise ValueError("samples must be a contiguous int64 CUDA tensor of at least 6 elements")
     n = samples.numel()
     return load().streamkl_probe_clock(int(duration_ns), int(interval_ns), _ptr(samples),
                                        int((n - 2) // 2), _stream(stream))

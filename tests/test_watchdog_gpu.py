@@ -81,6 +81,10 @@ def test_clock_probe_reads_a_plausible_clock_beside_a_kernel():
     kl, l1, l2 = (torch.empty((w.B, w.Hq, w.NQ), device="cuda") for _ in range(3))
     samples = torch.zeros(2 + 2 * 400, dtype=torch.int64, device="cuda")
     side = torch.cuda.Stream()
+    for bad in (torch.zeros(800, dtype=torch.float32, device="cuda"),
+                torch.zeros(4, dtype=torch.int64, device="cuda"), torch.zeros(800, dtype=torch.int64)):
+        with pytest.raises(ValueError):
+            binding.streamkl_probe_clock(20_000_000, 100_000, bad, side)
     assert binding.streamkl_probe_clock(20_000_000, 100_000, samples, side) == binding.OK
     for _ in range(5):
         binding.fwd(t["q1"], t["k1"], t["q2"], t["k2"], scale=w.scale, causal=True, out=(kl, l1, l2))
