@@ -35,6 +35,11 @@ CASES = [
     (1, 2, 2, 300, 1000, 128, False, False, 4),    # two query tiles per block, ragged rows
     (1, 2, 2, 700, 700, 128, True, True, 3),       # causal: early blocks own empty ranges
     (1, 1, 1, 5, 1, 128, False, True, 8),          # one key: one range, no workspace
+    # row counts at the layout boundaries: 9 (first past the keys-as-rows kernel), 32 (the
+    # last with rows copied into all four lane quarters), 33 (one 128-row query tile)
+    (1, 2, 2, 9, 2000, 128, False, True, 0),
+    (1, 2, 2, 32, 1500, 64, False, False, 3),
+    (1, 2, 2, 33, 1500, 128, False, True, 2),
 ]
 
 
