@@ -125,11 +125,13 @@ size_t streamkl_fwd_splitk_workspace_bytes(int B, int Hq, int NQ, int NK, int sp
 /*
  * Bytes of fp32 workspace streamkl_bwd needs for these sizes: the dK accumulator,
  * B*Hkv*ceil(NK/128)*128*d*4 (whole 128-row key tiles), plus, when streamkl_bwd splits each
- * query tile's keys into ranges (its B*Hq*ceil(NQ/128) query tiles alone would leave SMs
- * idle and there are at least two key tiles), the dQ partial sums
- * B*Hq*ceil(NQ/128)*128*d*4.  Returns 0 for sizes outside the supported range.  The split
- * decision depends on the SM count of the current device (streamkl_num_sms), so query with
- * the device current that the backward will run on.
+ * query tile's keys into ranges (its CTAs alone would leave SMs idle and there are at least
+ * two key tiles), the dQ partial sums B*Hq*ceil(NQ/128)*128*d*4.  The backward runs one CTA
+ * per query tile and query head, or per query tile and pair of query heads when d = 64 and
+ * Hq/Hkv is even, so B*Hq*ceil(NQ/128) or half that CTAs before any split.  Returns 0 for
+ * sizes outside the supported range.  The split decision depends on the SM count of the
+ * current device (streamkl_num_sms), so query with the device current that the backward will
+ * run on.
  */
 size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int d);
 
@@ -145,7 +147,9 @@ size_t streamkl_bwd_workspace_bytes(int B, int Hq, int Hkv, int NQ, int NK, int 
  *   share the KV head.  The fixed distribution gets no gradient; with k1 == k2 the
  *   returned dk is the gradient through the free distribution only.
  * One CTA owns a 128-row query tile and visits every key tile its rows see, once ("Fusão de
- * Kernel").  When those CTAs alone would leave SMs idle (few query rows, long keys), each
+ * Kernel"); at d = 64 with an even number of query heads per KV head it owns that tile in two
+ * heads of one group, and their dK partials meet on chip.  When those CTAs alone would leave
+ * SMs idle (few query rows, long keys), each
  * tile's keys are split into ranges handled by separate CTAs and dQ is summed through the
  * workspace too; the choice is the library's and is reflected in
  * streamkl_bwd_workspace_bytes.  Launches: a workspace memset, the backward kernel, one
