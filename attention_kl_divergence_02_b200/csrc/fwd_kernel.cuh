@@ -606,6 +606,9 @@ streamkl_fwd_kernel(const __grid_constant__ CUtensorMap tmQ1, const __grid_const
 __global__ void __launch_bounds__(256)
 streamkl_splitk_merge_kernel(const float* __restrict__ part, int splits, long long R, float scale,
                              float* __restrict__ kl, float* __restrict__ lse1, float* __restrict__ lse2) {
+    // launched as a programmatic dependent of the forward: wait until that grid has completed
+    // and its partial states are visible (no-op when launched without the dependency)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (long long o = blockIdx.x * (long long)blockDim.x + threadIdx.x; o < R;
          o += (long long)gridDim.x * blockDim.x) {
         float M1 = -1e30f, M2 = -1e30f;

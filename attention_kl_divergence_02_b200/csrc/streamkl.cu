@@ -285,6 +285,27 @@ void split_ranges(int NK, int splits, int* kps, int* used) {
     *used = (nkt + *kps - 1) / *kps;
 }
 
+// The split-K merge, launched as a programmatic dependent of the forward kernel just queued on
+// the same stream: its launch and ramp overlap that grid's last CTAs, and its first
+// instruction waits until the forward grid has completed and its partial states are visible.
+int launch_merge(const float* part, int splits, long long R, float scale, float* kl, float* lse1,
+                 float* lse2, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<long long>((R + 255) / 256, 8ll * num_sms()));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, skl::streamkl_splitk_merge_kernel, part, splits, R, scale,
+                                       kl, lse1, lse2);
+    if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+    return STREAMKL_OK;
+}
+
 // kl21 != nullptr: the symmetric variant (also KL(P2 || P1) per row), one key range only.
 int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const uint16_t* k2, int B,
              int Hq, int Hkv, int NQ, int NK, int d, float scale, int causal, int splits, float* kl,
@@ -320,12 +341,7 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
                         : launch_fwd_keys_rows<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
         }
         if (rc || p.splits == 1) return rc;
-        const long long R = (long long)B * Hq * NQ;
-        const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * num_sms());
-        skl::streamkl_splitk_merge_kernel<<<mgrid, 256, 0, st>>>(part, p.splits, R, scale, kl, lse1, lse2);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
-        return STREAMKL_OK;
+        return launch_merge(part, p.splits, (long long)B * Hq * NQ, scale, kl, lse1, lse2, st);
     }
     // at most 32 query rows: they are loaded once into each 32-lane quarter of the query
     // tile (32-row boxes), so that all four warps of a warpgroup can fold them
@@ -355,12 +371,7 @@ int fwd_impl(const uint16_t* q1, const uint16_t* k1, const uint16_t* q2, const u
                     : launch_fwd<64, false>(mq1, mq2, mk1, mk2, p, (int)grid, st);
     }
     if (rc || p.splits == 1) return rc;
-    const long long R = (long long)B * Hq * NQ;
-    const int mgrid = (int)std::min<long long>((R + 255) / 256, 8ll * num_sms());
-    skl::streamkl_splitk_merge_kernel<<<mgrid, 256, 0, st>>>(part, p.splits, R, scale, kl, lse1, lse2);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
-    return STREAMKL_OK;
+    return launch_merge(part, p.splits, (long long)B * Hq * NQ, scale, kl, lse1, lse2, st);
 }
 
 }  // namespace
