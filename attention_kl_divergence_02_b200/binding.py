@@ -39,6 +39,7 @@ EXPORTS = (
     "streamkl_probe_exp2",
     "streamkl_num_sms",
     "streamkl_probe_clock",
+    "streamkl_eval_exp2",
 )
 
 _lib = None
@@ -98,6 +99,8 @@ def load(path=None):
     lib.streamkl_num_sms.restype = i
     lib.streamkl_probe_clock.argtypes = [ctypes.c_longlong, ctypes.c_longlong, vp, i, vp]
     lib.streamkl_probe_clock.restype = i
+    lib.streamkl_eval_exp2.argtypes = [i, vp, vp, ctypes.c_longlong, vp]
+    lib.streamkl_eval_exp2.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -211,6 +214,17 @@ def streamkl_probe_clock(duration_ns, interval_ns, samples, stream=None):
     n = samples.numel()
     return load().streamkl_probe_clock(int(duration_ns), int(interval_ns), _ptr(samples),
                                        int((n - 2) // 2), _stream(stream))
+
+
+def streamkl_eval_exp2(kind, x, stream=None):
+    """2^x by the kernels' exponential path `kind` (0: exponential unit, 1: FMA-pipe
+    polynomial) for a contiguous fp32 CUDA tensor; returns (status, y)."""
+    import torch
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    rc = load().streamkl_eval_exp2(int(kind), _ptr(x), _ptr(y), x.numel(), _stream(stream))
+    return rc, y
 
 
 def status_string(status):

@@ -46,6 +46,20 @@ streamkl_probe_exp2_kernel(int iters, int write, float* sink) {
     if (write) sink[blockIdx.x * kProbeThreads + threadIdx.x] = s;
 }
 
+// y[i] = 2^x[i] by one of the kernels' two exponential paths (KIND 0: ex2.approx on the
+// exponential unit; 1: the FMA-pipe polynomial ex2_poly2), for checking their accuracy.
+template <int KIND>
+__global__ void __launch_bounds__(256)
+streamkl_eval_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+    for (long long i = 2 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < n;
+         i += 2 * (long long)gridDim.x * blockDim.x) {
+        const float2 u = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+        const float2 e = KIND == 0 ? make_float2(ex2(u.x), ex2(u.y)) : ex2_poly2(u);
+        y[i] = e.x;
+        if (i + 1 < n) y[i + 1] = e.y;
+    }
+}
+
 // Effective SM clock.  Under the board's power cap the SM clock drops below its maximum for
 // as long as heavy kernels run, and a sampled clock reading can miss it; clock64 counts the
 // cycles an SM actually runs.  One thread records (globaltimer ns, clock64) pairs every

@@ -243,25 +243,14 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x for x <= 0 on the FMA/ALU pipes, so part of a kernel's exponentials can run beside
-// the exponential unit.  Range reduction x = j + f with j = round(x) (adding and removing
-// 1.5*2^23 rounds to an integer), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial fitted
-// for minimax relative error with the Remez exchange (fit_exp2_poly.py beside this file;
-// worst relative error 2.7e-6 in fp32); 2^j applied by adding j to the exponent field
-// (the low bits of the rounded sum hold j).  x is clamped at -126, so the result is
-// >= 0 and tiny instead of wrapping; -inf gives about 1e-38.
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(9.570102207e-03f, f, 5.591785908e-02f);
-    p = fmaf(p, f, 2.402474433e-01f);
-    p = fmaf(p, f, 6.931217909e-01f);
-    p = fmaf(p, f, 9.999992847e-01f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// ex2_poly on two values at once with packed fp32x2 arithmetic (one instruction per pair).
+// 2^x for x <= 0 on the FMA/ALU pipes, two values at once with packed fp32x2 arithmetic (one
+// instruction per pair), so part of a kernel's exponentials can run beside the exponential
+// unit.  Range reduction x = j + f with j = round(x) (adding and removing 1.5*2^23 rounds to an
+// integer), f in [-1/2, 1/2]; 2^f by a degree-4 polynomial fitted for minimax relative error
+// with the Remez exchange (fit_exp2_poly.py beside this file; worst relative error 2.7e-6 in
+// fp32); 2^j applied by adding j to the exponent field (the low bits of the rounded sum hold
+// j).  x is clamped at -126, so the result is >= 0 and tiny instead of wrapping; -inf gives
+// about 1e-38.
 __device__ __forceinline__ float2 ex2_poly2(float2 u) {
     u.x = fmaxf(u.x, -126.0f);
     u.y = fmaxf(u.y, -126.0f);

@@ -258,6 +258,20 @@ int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream) {
 
 int streamkl_num_sms(void) { return num_sms(); }
 
+int streamkl_eval_exp2(int kind, const float* x, float* y, long long n, void* stream) {
+    if ((kind != 0 && kind != 1) || n < 0 || (n > 0 && (!x || !y))) return STREAMKL_ERR_INVALID_ARG;
+    if (n == 0) return STREAMKL_OK;
+    const long long blocks = std::min<long long>((n + 511) / 512, 8ll * num_sms());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == 0)
+        skl::streamkl_eval_exp2_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(x, y, n);
+    else
+        skl::streamkl_eval_exp2_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(x, y, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "exp2 evaluation launch");
+    return STREAMKL_OK;
+}
+
 int streamkl_probe_clock(long long duration_ns, long long interval_ns, long long* samples,
                          int max_pairs, void* stream) {
     if (!samples) return STREAMKL_ERR_INVALID_ARG;

@@ -228,6 +228,17 @@ int streamkl_probe_exp2(int kind, int iters, long long* n_exp, void* stream);
 int streamkl_num_sms(void);
 
 /*
+ * y[i] = 2^x[i] for i < n by one of the two exponential paths the kernels use, for checking
+ * their accuracy; no part of the KL computation.  kind 0: ex2.approx on the exponential unit
+ * (subnormal results flushed to zero); kind 1: the FMA-pipe polynomial (x clamped at -126,
+ * worst relative error of the fit 2.7e-6 for -126 <= x <= 0; meant for x <= 0).
+ *   x, y : device arrays of n fp32 (caller-owned; y may not overlap x).
+ * One kernel on `stream`.  Returns STREAMKL_ERR_INVALID_ARG for a bad kind, n < 0 or a NULL
+ * array with n > 0; n = 0 launches nothing.
+ */
+int streamkl_eval_exp2(int kind, const float* x, float* y, long long n, void* stream);
+
+/*
  * Effective SM clock probe; no part of the KL computation.  Under the board's power cap
  * the SM clock runs below its maximum while heavy kernels run, so a kernel's time depends
  * on that clock; this records it while other work runs.  Launches one 32-thread CTA on
