@@ -53,6 +53,7 @@ CASES = [
     (1, 4, 2, 333, 333, 64, True, False),
     (1, 8, 2, 257, 257, 64, True, True),
     (2, 4, 2, 130, 1000, 64, False, False),
+    (1, 8, 1, 200, 700, 64, False, False),     # 8:1: four head pairs share one KV head
 ]
 
 
