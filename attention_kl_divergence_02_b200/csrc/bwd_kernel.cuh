@@ -29,6 +29,11 @@
 // MMAs of visit n still read theirs, so the tensor core is handed work without waiting for
 // the write.
 //
+// At d = 64, when a KV group has an even number of query heads (HP = 2), a CTA owns the same
+// query tile of two heads of the group: visits alternate between the heads for each key tile
+// (loaded once), each head's dQ has its own TMEM columns, and the dK partial of a key tile
+// sums both heads' visits before one flush.
+//
 // When the query tiles alone would leave SMs idle, the library splits each tile's key tiles
 // into ranges (one CTA each); dQ is then added into a second tile-blocked fp32 workspace
 // instead of being written once, and converted like dK.
