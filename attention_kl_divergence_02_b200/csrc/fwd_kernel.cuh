@@ -28,7 +28,11 @@
 // with splits > 1 the key tiles are cut into ranges of kps tiles, CTA (block, split) folds
 // only its range, and instead of finishing it stores the five scalars of each row; the
 // merge kernel below combines the ranges exactly (each rescaled to the common maximum, the
-// same correction the online recurrence applies tile by tile).
+// same correction the online recurrence applies tile by tile).  The merge is launched as a
+// programmatic dependent of this kernel and waits for it with griddepcontrol.wait.
+//
+// At most 8 query rows run in fwd_keys_kernel.cuh instead (keys as the MMA's rows); the
+// symmetric variant (SYM) adds the reverse direction's running sum to either kernel.
 #pragma once
 
 #include "sm100.cuh"
