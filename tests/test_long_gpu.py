@@ -7,7 +7,10 @@ to fp64 on its own:
   * KL, LSE1, LSE2 and dQ (P1 fixed) on sampled rows, from the oracle's own row statistics;
   * dK on sampled keys, from the GPU's row statistics (KL, LSE1, LSE2 of all 65536 rows
     of the head -- too many for the fp64 oracle), which the first check spot-verifies: that
-    part of the check is only partly independent.
+    part of the check is only partly independent;
+  * dK on keys among the last 256, fully independent: under the causal mask only the last
+    256 rows see them, so the oracle computes those rows' statistics itself and every other
+    row's statistics are NaN (any use of them would show).
 """
 import numpy as np
 import pytest
@@ -49,5 +52,16 @@ def test_long64k_forward_and_mode1_backward_sampled():
         odk = oracle.bwd_dk_keys_stats(1, q1, k, q2, k, g, *stats, keys, scale=w.scale, causal=True)
         gdk = dk[0, h].float().cpu().double().numpy()[keys]
         assert rel_l2(gdk[None, None], odk[None, None], axes=(2, 3)).max() <= GRAD_TOL
+        # the last keys: seen only by the last 256 rows, whose statistics the oracle computes
+        tail = np.arange(N - 256, N)
+        tkl, tl1, tl2 = oracle.fwd_rows(q1, k, q2, k, tail, scale=w.scale, causal=True)
+        own = [np.full((1, 1, N), np.nan) for _ in range(3)]
+        for a, v in zip(own, (tkl, tl1, tl2)):
+            a[0, 0, tail] = v
+        last = np.array([N - 256, N - 200, N - 129, N - 128, N - 17, N - 1])
+        odk2 = oracle.bwd_dk_keys_stats(1, q1, k, q2, k, g, *own, last, scale=w.scale, causal=True)
+        assert np.all(np.isfinite(odk2))
+        gdk2 = dk[0, h].float().cpu().double().numpy()[last]
+        assert rel_l2(gdk2[None, None], odk2[None, None], axes=(2, 3)).max() <= GRAD_TOL
     assert bool(torch.isfinite(kl).all()) and bool(torch.isfinite(dq.float()).all())
     assert kl.min().item() >= -2e-3
